@@ -1,0 +1,178 @@
+"""Python access to the C oracle (``oracle/dg_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke()`` and by the
+benchmark's CPU-baseline / reference leg. The library's product path never imports it.
+
+All arrays are numpy; bf16 values travel as their uint16 bit patterns and e4m3 values as
+their uint8 codes. Results of the GEMMs are fp64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dg_oracle.c")
+_LIB = os.path.join(_HERE, "libdg_oracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compiles the oracle with gcc (fp-contract off, no fast-math, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+                               "-ffp-contract=off", "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P, I, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+        L.dgo_e4m3_decode.restype = D
+        L.dgo_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.dgo_e4m3_encode_satrne.restype = ctypes.c_uint8
+        L.dgo_e4m3_encode_satrne.argtypes = [ctypes.c_float]
+        L.dgo_bf16_to_f32.restype = ctypes.c_float
+        L.dgo_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.dgo_cast_per_token.argtypes = [P, I, I, P, P]
+        L.dgo_cast_per_block.argtypes = [P, I, I, I, P, P]
+        L.dgo_transform_sf.argtypes = [P, I, I, I, P]
+        L.dgo_gemm_nt.argtypes = [P, P, P, P, P, I, I, I, P, I, P]
+        L.dgo_m_grouped_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, P]
+        L.dgo_m_grouped_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
+        for f in ("dgo_cast_per_token", "dgo_cast_per_block", "dgo_transform_sf", "dgo_gemm_nt",
+                  "dgo_m_grouped_contiguous", "dgo_m_grouped_masked", "dgo_num_threads"):
+            getattr(L, f).restype = I
+        _lib = L
+    return _lib
+
+
+def _p(arr):
+    return None if arr is None else arr.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(arr, dtype):
+    return None if arr is None else np.ascontiguousarray(arr, dtype=dtype)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (code {rc})")
+
+
+def pad4(x: int) -> int:
+    return (x + 3) // 4 * 4
+
+
+def num_threads() -> int:
+    return lib().dgo_num_threads()
+
+
+def e4m3_decode(code: int) -> float:
+    return lib().dgo_e4m3_decode(int(code))
+
+
+def e4m3_encode(y: float) -> int:
+    return lib().dgo_e4m3_encode_satrne(float(y))
+
+
+def e4m3_table() -> np.ndarray:
+    """fp64 value of every e4m3 code (NaN for the two NaN codes)."""
+    return np.array([e4m3_decode(c) for c in range(256)], dtype=np.float64)
+
+
+def cast_per_token(x_bf16: np.ndarray):
+    """x [M,K] bf16 bits -> (q [M,K] uint8, sfa [Kb, pad4(M)] fp32; padding entries 0)."""
+    x = _c(x_bf16, np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), np.uint8)
+    sfa = np.zeros((K // 128, pad4(M)), np.float32)
+    _check(lib().dgo_cast_per_token(_p(x), M, K, _p(q), _p(sfa)), "cast_per_token")
+    return q, sfa
+
+
+def cast_per_block(x_bf16: np.ndarray):
+    """x [N,K] or [G,N,K] bf16 bits -> (q same shape, sfb [G?, ceil(N/128), Kb] fp32)."""
+    x = _c(x_bf16, np.uint16)
+    squeeze = x.ndim == 2
+    if squeeze:
+        x = x[None]
+    G, N, K = x.shape
+    q = np.empty((G, N, K), np.uint8)
+    sfb = np.empty((G, (N + 127) // 128, K // 128), np.float32)
+    _check(lib().dgo_cast_per_block(_p(x), G, N, K, _p(q), _p(sfb)), "cast_per_block")
+    return (q[0], sfb[0]) if squeeze else (q, sfb)
+
+
+def transform_sf(sf_kmajor: np.ndarray) -> np.ndarray:
+    """[MN, Kb] or [B, MN, Kb] fp32 -> [Kb, pad4(MN)] or [B, Kb, pad4(MN)] (tail zero)."""
+    s = _c(sf_kmajor, np.float32)
+    squeeze = s.ndim == 2
+    if squeeze:
+        s = s[None]
+    B, MN, Kb = s.shape
+    out = np.empty((B, Kb, pad4(MN)), np.float32)
+    _check(lib().dgo_transform_sf(_p(s), B, MN, Kb, _p(out)), "transform_sf")
+    return out[0] if squeeze else out
+
+
+def gemm_nt(a, sfa, b, sfb, c=None, rows=None) -> np.ndarray:
+    """fp64 D (or the listed rows of D) for the dense block-scaled NT GEMM."""
+    a = _c(a, np.uint8); b = _c(b, np.uint8)
+    sfa = _c(sfa, np.float32); sfb = _c(sfb, np.float32); c = _c(c, np.uint16)
+    M, K = a.shape
+    N = b.shape[0]
+    assert sfa.shape == (K // 128, pad4(M)), sfa.shape
+    assert sfb.shape == ((N + 127) // 128, K // 128), sfb.shape
+    r = None if rows is None else _c(rows, np.int32)
+    R = M if r is None else r.shape[0]
+    out = np.empty((R, N), np.float64)
+    _check(lib().dgo_gemm_nt(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), M, N, K, _p(r), R, _p(out)),
+           "gemm_nt")
+    return out
+
+
+def m_grouped_contiguous(a, sfa, b, sfb, grouped_layout, c=None, rows=None) -> np.ndarray:
+    a = _c(a, np.uint8); b = _c(b, np.uint8)
+    sfa = _c(sfa, np.float32); sfb = _c(sfb, np.float32); c = _c(c, np.uint16)
+    gl = _c(grouped_layout, np.int32)
+    M_sum, K = a.shape
+    G, N, _ = b.shape
+    r = None if rows is None else _c(rows, np.int32)
+    R = M_sum if r is None else r.shape[0]
+    out = np.empty((R, N), np.float64)
+    _check(lib().dgo_m_grouped_contiguous(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(gl), M_sum, N, K,
+                                          G, _p(r), R, _p(out)), "m_grouped_contiguous")
+    return out
+
+
+def m_grouped_masked(a, sfa, b, sfb, masked_m, c=None) -> np.ndarray:
+    a = _c(a, np.uint8); b = _c(b, np.uint8)
+    sfa = _c(sfa, np.float32); sfb = _c(sfb, np.float32); c = _c(c, np.uint16)
+    mm = _c(masked_m, np.int32)
+    G, M_max, K = a.shape
+    N = b.shape[1]
+    out = np.empty((G, M_max, N), np.float64)
+    _check(lib().dgo_m_grouped_masked(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(mm), G, M_max, N, K,
+                                      _p(out)), "m_grouped_masked")
+    return out
+
+
+def tolerance_ok(d: np.ndarray, ref: np.ndarray, rel: float = 2.0 ** -7, abs_rms: float = 1e-2):
+    """Per-element bound |D - ref| <= rel·|ref| + abs_rms·rms(ref); returns (ok, worst ratio)."""
+    ref = np.asarray(ref, np.float64)
+    d = np.asarray(d, np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    bound = rel * np.abs(ref) + abs_rms * rms
+    err = np.abs(d - ref)
+    ratio = float(np.max(err / np.maximum(bound, 1e-300))) if ref.size else 0.0
+    return bool(np.all(err <= bound)), ratio

@@ -1,0 +1,292 @@
+/*
+ * dg_oracle.c — plain, slow, exact CPU oracle for the FP8 block-scaled NT GEMM.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the library's product path links, loads or calls this
+ * file; only the tests, the smoke check and the benchmark's CPU-baseline leg do. It shares no
+ * code, header, table or constant with the CUDA library.
+ *
+ * Pages cited (the DeepGEMM write-ups this library is built from):
+ *   [likun]   likun.im/craft/deepgemm — "DeepGEMM 一句话"; §一 (what it is: D = C + A·Bᵀ in NT
+ *             layout, M-grouped contiguous / masked), §二 (the register_apis list), §五 (the
+ *             scale-factor layout caveat: the LHS scales need a TMA-aligned transposed layout).
+ *   [aitang]  aitangshan.cn/news/1491278 — §5 "平台核心功能" (grouped GEMM: contiguous and masked
+ *             layouts) and 技术原理 §4 "FP8 精度优化的核心" (block-wise scaling: one scale per
+ *             block, the product restored by the scale after the multiplication).
+ *   [zwt]     zwt0204.github.io "DeepGEMM deep dive" — §"它的核心思路" (grouped layout
+ *             constraint; masked layout for decoding).
+ *   [OCP]     OCP 8-bit Floating Point Specification (OFP8) rev 1.0, format E4M3: bias 7,
+ *             no infinities, S.1111.111 is NaN, largest finite 448, subnormal step 2^-9.
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - cast scale s = amax / 448 (fp32, correctly rounded); amax == 0 gives s = 1;
+ *   - the value is divided by the scale (y = x / s, fp32 correctly rounded), not multiplied
+ *     by a reciprocal;
+ *   - y is rounded to nearest-even onto the E4M3 grid (subnormals included) and then clamped
+ *     to ±448 with its sign kept; a zero keeps its sign (-0 encodes as 0x80);
+ *   - a partial 128-row weight block (N not a multiple of 128) takes amax over its valid rows;
+ *   - "multiply by the scale after the GEMM" is applied per 128-wide K block:
+ *       D[m,n] = C[m,n] + sum_kb sfa[m,kb]·sfb[n/128,kb]·S_kb[m,n],
+ *       S_kb[m,n] = sum_{k in kb} e4m3(A[m,k])·e4m3(B[n,k]);
+ *     every S_kb is exact in fp64 (each product is a multiple of 2^-18 below 2^17.6 and 128 of
+ *     them need at most 43 significant bits), so the only rounding is in the fp64 scale sum;
+ *   - sfa layout: fp32 [Kb][pad4(M)] (MN-major, rows padded to a multiple of 4 so each K-block
+ *     row starts 16-byte aligned); sfb layout: fp32 [G][ceil(N/128)][Kb];
+ *   - masked rows r >= masked_m[g] are never written; contiguous padding rows (-1) have no
+ *     defined value.
+ *
+ * All entry points return 0 on success and a negative value on bad arguments.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define DGO_BLK 128
+
+static int pad4(int x) { return (x + 3) / 4 * 4; }
+
+/* ---------------------------------------------------------------------------------------- */
+/* Number formats                                                                            */
+/* ---------------------------------------------------------------------------------------- */
+
+/* [OCP] E4M3 decode: exponent field e (4 bits), mantissa m (3 bits), bias 7.
+ * e == 0 -> subnormal m * 2^-9; otherwise (1 + m/8) * 2^(e-7); S.1111.111 -> NaN. */
+double dgo_e4m3_decode(uint8_t code) {
+    int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* [OCP] E4M3 encode of a finite fp32 value with round-to-nearest-even, then saturation to
+ * the largest finite magnitude 448 (sign kept). Works on the exact value in double. */
+uint8_t dgo_e4m3_encode_satrne(float y) {
+    uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    double a = fabs((double)y);
+    if (a >= 448.0) return sign | 0x7E;              /* 448 = 1.75 * 2^8: e=15, m=6 */
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal range: grid step 2^-9, codes 0..8 map to n * 2^-9 (8 is the smallest normal) */
+        double n = nearbyint(ldexp(a, 9));          /* exact scaling; ties to even */
+        return sign | (uint8_t)n;
+    }
+    int e;
+    frexp(a, &e);                                   /* a = f * 2^e, f in [0.5, 1) */
+    e -= 1;                                         /* a in [2^e, 2^(e+1)) */
+    /* grid step at this binade is 2^(e-3); n in [8, 16] after rounding */
+    double n = nearbyint(ldexp(a, 3 - e));
+    int code = ((e + 7) << 3) + ((int)n - 8);       /* n == 16 carries into the next binade */
+    return sign | (uint8_t)code;
+}
+
+/* bf16 is the upper half of an IEEE binary32 pattern. */
+float dgo_bf16_to_f32(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* ---------------------------------------------------------------------------------------- */
+/* Casts (block-wise scaling: [aitang] 技术原理 §4)                                          */
+/* ---------------------------------------------------------------------------------------- */
+
+static float scale_from_amax(float amax) {
+    if (amax == 0.0f) return 1.0f;
+    return amax / 448.0f;                           /* IEEE fp32 division */
+}
+
+/* Per-token cast: for every row m and 128-wide K slice kb,
+ *   amax = max |x[m, kb*128 .. kb*128+127]|,  s = amax/448,  q = e4m3_satrne(x / s),
+ * with sfa written MN-major: sfa[kb * pad4(M) + m] = s. Padding entries are left untouched.
+ * x: bf16 bits [M,K]; q: [M,K]; K must be a multiple of 128. */
+int dgo_cast_per_token(const uint16_t *x, int M, int K, uint8_t *q, float *sfa) {
+    if (M < 0 || K <= 0 || K % DGO_BLK) return -1;
+    int Kb = K / DGO_BLK, ld = pad4(M);
+#pragma omp parallel for schedule(static)
+    for (int m = 0; m < M; m++) {
+        for (int kb = 0; kb < Kb; kb++) {
+            const uint16_t *xs = x + (size_t)m * K + (size_t)kb * DGO_BLK;
+            float amax = 0.0f;
+            for (int i = 0; i < DGO_BLK; i++) {
+                float v = fabsf(dgo_bf16_to_f32(xs[i]));
+                if (v > amax) amax = v;
+            }
+            float s = scale_from_amax(amax);
+            for (int i = 0; i < DGO_BLK; i++)
+                q[(size_t)m * K + (size_t)kb * DGO_BLK + i] = dgo_e4m3_encode_satrne(dgo_bf16_to_f32(xs[i]) / s);
+            sfa[(size_t)kb * ld + m] = s;
+        }
+    }
+    return 0;
+}
+
+/* Per-block cast of weights: for every batch g, 128-row block nb and K slice kb,
+ * amax over rows [nb*128, min(N, nb*128+128)) and the slice's 128 columns; then as above.
+ * x: bf16 bits [batch,N,K]; q: [batch,N,K]; sfb: [batch][ceil(N/128)][Kb]. */
+int dgo_cast_per_block(const uint16_t *x, int batch, int N, int K, uint8_t *q, float *sfb) {
+    if (batch < 0 || N < 0 || K <= 0 || K % DGO_BLK) return -1;
+    int Kb = K / DGO_BLK, Nb = (N + DGO_BLK - 1) / DGO_BLK;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int g = 0; g < batch; g++) {
+        for (int nb = 0; nb < Nb; nb++) {
+            int n_end = (nb + 1) * DGO_BLK < N ? (nb + 1) * DGO_BLK : N;
+            for (int kb = 0; kb < Kb; kb++) {
+                float amax = 0.0f;
+                for (int n = nb * DGO_BLK; n < n_end; n++)
+                    for (int i = 0; i < DGO_BLK; i++) {
+                        float v = fabsf(dgo_bf16_to_f32(x[((size_t)g * N + n) * K + (size_t)kb * DGO_BLK + i]));
+                        if (v > amax) amax = v;
+                    }
+                float s = scale_from_amax(amax);
+                for (int n = nb * DGO_BLK; n < n_end; n++)
+                    for (int i = 0; i < DGO_BLK; i++) {
+                        size_t off = ((size_t)g * N + n) * K + (size_t)kb * DGO_BLK + i;
+                        q[off] = dgo_e4m3_encode_satrne(dgo_bf16_to_f32(x[off]) / s);
+                    }
+                sfb[((size_t)g * Nb + nb) * Kb + kb] = s;
+            }
+        }
+    }
+    return 0;
+}
+
+/* Scale-layout transform ([likun] §五: LHS scales in a TMA-aligned transposed layout):
+ * in  fp32 [batch][MN][Kb]  (K-major, one row of Kb scales per token)
+ * out fp32 [batch][Kb][pad4(MN)] (MN-major); the pad4 tail of each row is set to 0. */
+int dgo_transform_sf(const float *in, int batch, int MN, int Kb, float *out) {
+    if (batch < 0 || MN < 0 || Kb < 0) return -1;
+    int ld = pad4(MN);
+    for (int b = 0; b < batch; b++)
+        for (int kb = 0; kb < Kb; kb++)
+            for (int i = 0; i < ld; i++)
+                out[((size_t)b * Kb + kb) * ld + i] = i < MN ? in[((size_t)b * MN + i) * Kb + kb] : 0.0f;
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------------- */
+/* GEMM: D = C + A·Bᵀ, NT ([likun] §一), block-scaled ([aitang] 技术原理 §4)                 */
+/* ---------------------------------------------------------------------------------------- */
+
+/* One output element: C + sum_kb (sfa·sfb)·S_kb with S_kb summed exactly in fp64.
+ * arow, brow: e4m3 codes of length K; sfa_row(kb) = sfa_base[kb * sfa_ld];
+ * sfb_row(kb) = sfb_base[kb]. */
+static double dot_row(const uint8_t *arow, const float *sfa_base, size_t sfa_ld,
+                      const uint8_t *brow, const float *sfb_base, int Kb, const double *lut) {
+    double acc = 0.0;
+    for (int kb = 0; kb < Kb; kb++) {
+        double s = 0.0;
+        const uint8_t *ap = arow + (size_t)kb * DGO_BLK, *bp = brow + (size_t)kb * DGO_BLK;
+        for (int i = 0; i < DGO_BLK; i++) s += lut[ap[i]] * lut[bp[i]];
+        double scale = (double)sfa_base[(size_t)kb * sfa_ld] * (double)sfb_base[kb];
+        acc += scale * s;
+    }
+    return acc;
+}
+
+static void fill_lut(double *lut) {
+    for (int c = 0; c < 256; c++) lut[c] = dgo_e4m3_decode((uint8_t)c);
+}
+
+/* Dense: A e4m3 [M,K], sfa [Kb][pad4(M)], B e4m3 [N,K], sfb [ceil(N/128)][Kb],
+ * C bf16 [M,N] or NULL. Computes the rows listed in `rows` (all rows when rows == NULL,
+ * nrows is then ignored) into out[nrows or M][N] as fp64. */
+int dgo_gemm_nt(const uint8_t *a, const float *sfa, const uint8_t *b, const float *sfb,
+                const uint16_t *c, int M, int N, int K, const int *rows, int nrows, double *out) {
+    if (M < 0 || N < 0 || K <= 0 || K % DGO_BLK) return -1;
+    int Kb = K / DGO_BLK, R = rows ? nrows : M;
+    size_t ld = (size_t)pad4(M);
+    double lut[256];
+    fill_lut(lut);
+    for (int r = 0; r < R; r++) if (rows && (rows[r] < 0 || rows[r] >= M)) return -2;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < R; r++) {
+        int m = rows ? rows[r] : r;
+        for (int n = 0; n < N; n++) {
+            double v = dot_row(a + (size_t)m * K, sfa + m, ld, b + (size_t)n * K,
+                               sfb + (size_t)(n / DGO_BLK) * Kb, Kb, lut);
+            if (c) v += (double)dgo_bf16_to_f32(c[(size_t)m * N + n]);
+            out[(size_t)r * N + n] = v;
+        }
+    }
+    return 0;
+}
+
+/* M-grouped contiguous ([likun] §二 m_grouped_*_contiguous with grouped_layout; [zwt]):
+ * row r of A [M_sum,K] belongs to expert g = grouped_layout[r]; -1 marks a padding row.
+ * D[r] = C[r] + A[r]·B[g]ᵀ with B [G,N,K], sfb [G][ceil(N/128)][Kb], sfa [Kb][pad4(M_sum)].
+ * Padding rows get NaN in `out` (no defined value). rows/nrows as in dgo_gemm_nt. */
+int dgo_m_grouped_contiguous(const uint8_t *a, const float *sfa, const uint8_t *b, const float *sfb,
+                             const uint16_t *c, const int32_t *grouped_layout, int M_sum, int N, int K,
+                             int G, const int *rows, int nrows, double *out) {
+    if (M_sum < 0 || N < 0 || K <= 0 || K % DGO_BLK || G <= 0) return -1;
+    int Kb = K / DGO_BLK, Nb = (N + DGO_BLK - 1) / DGO_BLK, R = rows ? nrows : M_sum;
+    size_t ld = (size_t)pad4(M_sum);
+    double lut[256];
+    fill_lut(lut);
+    for (int r = 0; r < R; r++) if (rows && (rows[r] < 0 || rows[r] >= M_sum)) return -2;
+    for (int m = 0; m < M_sum; m++) if (grouped_layout[m] >= G) return -3;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < R; r++) {
+        int m = rows ? rows[r] : r;
+        int g = grouped_layout[m];
+        for (int n = 0; n < N; n++) {
+            if (g < 0) { out[(size_t)r * N + n] = NAN; continue; }
+            const uint8_t *brow = b + ((size_t)g * N + n) * K;
+            const float *sfb_row = sfb + ((size_t)g * Nb + n / DGO_BLK) * Kb;
+            double v = dot_row(a + (size_t)m * K, sfa + m, ld, brow, sfb_row, Kb, lut);
+            if (c) v += (double)dgo_bf16_to_f32(c[(size_t)m * N + n]);
+            out[(size_t)r * N + n] = v;
+        }
+    }
+    return 0;
+}
+
+/* M-grouped masked ([likun] §二 m_grouped_*_masked with masked_m, expected_m; [zwt] masked
+ * layout for decoding): A [G,M_max,K], sfa [G][Kb][pad4(M_max)], B [G,N,K],
+ * sfb [G][ceil(N/128)][Kb], C [G,M_max,N] or NULL. For r < masked_m[g]:
+ * D[g,r] = C[g,r] + A[g,r]·B[g]ᵀ; rows r >= masked_m[g] are not part of the result and get
+ * NaN in `out` [G][M_max][N]. masked_m[g] is clamped to [0, M_max]. */
+int dgo_m_grouped_masked(const uint8_t *a, const float *sfa, const uint8_t *b, const float *sfb,
+                         const uint16_t *c, const int32_t *masked_m, int G, int M_max, int N, int K,
+                         double *out) {
+    if (G <= 0 || M_max < 0 || N < 0 || K <= 0 || K % DGO_BLK) return -1;
+    int Kb = K / DGO_BLK, Nb = (N + DGO_BLK - 1) / DGO_BLK;
+    size_t ld = (size_t)pad4(M_max);
+    double lut[256];
+    fill_lut(lut);
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int g = 0; g < G; g++) {
+        for (int m = 0; m < M_max; m++) {
+            int mm = masked_m[g] < 0 ? 0 : (masked_m[g] > M_max ? M_max : masked_m[g]);
+            double *orow = out + ((size_t)g * M_max + m) * N;
+            if (m >= mm) {
+                for (int n = 0; n < N; n++) orow[n] = NAN;
+                continue;
+            }
+            const uint8_t *arow = a + ((size_t)g * M_max + m) * K;
+            const float *sfa_base = sfa + (size_t)g * Kb * ld + m;
+            for (int n = 0; n < N; n++) {
+                const uint8_t *brow = b + ((size_t)g * N + n) * K;
+                const float *sfb_row = sfb + ((size_t)g * Nb + n / DGO_BLK) * Kb;
+                double v = dot_row(arow, sfa_base, ld, brow, sfb_row, Kb, lut);
+                if (c) v += (double)dgo_bf16_to_f32(c[((size_t)g * M_max + m) * N + n]);
+                orow[n] = v;
+            }
+        }
+    }
+    return 0;
+}
+
+int dgo_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
