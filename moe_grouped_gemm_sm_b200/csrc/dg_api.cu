@@ -1,0 +1,332 @@
+// dg_api.cu — the C ABI declared in include/dg.h: argument checks, TMA descriptor encoding,
+// tile-shape choice and kernel launch. No allocation, no synchronisation on the call path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dg.h"
+#include "dg_cast.cuh"
+#include "dg_gemm.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+__device__ int g_device_error;   // see dg_get_device_error()
+
+struct DeviceInfo {
+    bool ready = false;
+    int sm_count = 0;
+    int cc_major = 0, cc_minor = 0;
+    int *err = nullptr;          // device address of g_device_error
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+dg_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DG_OK : DG_ERR_CUDA; }
+
+// Per-device facts, queried once per device with that device current.
+dg_status device_info(const DeviceInfo **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DG_ERR_CUDA;
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!d.ready) {
+            if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DG_ERR_CUDA;
+            cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+            cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+            if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_device_error) != cudaSuccess) return DG_ERR_CUDA;
+            if (!g_encode) {
+                cudaDriverEntryPointQueryResult q;
+                void *fn = nullptr;
+                if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                    q != cudaDriverEntryPointSuccess || !fn)
+                    return DG_ERR_CUDA;
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            }
+            d.ready = true;
+        }
+    }
+    if (d.cc_major != 10 || d.cc_minor != 0) return DG_ERR_UNSUPPORTED;
+    *out = &d;
+    return DG_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int pad4(int x) { return (x + 3) / 4 * 4; }
+
+uint64_t wait_limit_ns() {
+    static std::atomic<uint64_t> cached{0};
+    uint64_t v = cached.load();
+    if (v == 0) {
+        v = 4000000000ull;   // 4 s per pipeline wait
+        if (const char *s = std::getenv("DG_WAIT_TIMEOUT_MS")) {
+            const long long ms = std::atoll(s);
+            if (ms > 0) v = static_cast<uint64_t>(ms) * 1000000ull;
+        }
+        cached.store(v);
+    }
+    return v;
+}
+
+// Encodes a tiled tensor map. dims/box are innermost first; strides (bytes) for dims 1..rank-1.
+bool encode(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
+            const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle sw) {
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    cuuint64_t d[5], s[4];
+    cuuint32_t b[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        if (i + 1 < rank) s[i] = strides[i];
+    }
+    const CUresult r = g_encode(m, dt, static_cast<cuuint32_t>(rank), const_cast<void *>(base), d, s, b, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct GemmMaps {
+    CUtensorMap a, b, sfa, c, d;
+};
+
+// Operand maps of one GEMM call. rows = rows of A/C/D per group; batched = 3D maps over G
+// groups for A, sfa, C and D (masked layout).
+template <int BN>
+bool build_maps(GemmMaps &mp, const void *a, const float *sfa, const void *b, const void *c, void *d,
+                int rows, int N, int K, int G, bool batched) {
+    const uint64_t Kb = static_cast<uint64_t>(K / 128);
+    const uint64_t ld = static_cast<uint64_t>(pad4(rows));
+    const uint64_t Gg = static_cast<uint64_t>(G);
+    {   // A: e4m3 [G?][rows][K], box 128 x 128, 128-byte swizzle
+        const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows), Gg};
+        const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(K) * rows};
+        const uint32_t box[3] = {128, 128, 1};
+        if (!encode(&mp.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, batched ? 3 : 2, a, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+            return false;
+    }
+    {   // B: e4m3 [G][N][K], box 128 x BN x 1
+        const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), Gg};
+        const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(K) * N};
+        const uint32_t box[3] = {128, BN, 1};
+        if (!encode(&mp.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return false;
+    }
+    {   // sfa: fp32 [G?][Kb][pad4(rows)], box 128 x 1
+        const uint64_t dims[3] = {ld, Kb, Gg};
+        const uint64_t str[2] = {ld * 4, ld * 4 * Kb};
+        const uint32_t box[3] = {128, 1, 1};
+        if (!encode(&mp.sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, batched ? 3 : 2, sfa, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+            return false;
+    }
+    {   // C, D: bf16 [G?][rows][N], box 64 x 32, 128-byte swizzle (one box row = 128 bytes)
+        const uint64_t dims[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(rows), Gg};
+        const uint64_t str[2] = {static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(N) * 2 * rows};
+        const uint32_t box[3] = {64, 32, 1};
+        if (!encode(&mp.d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, batched ? 3 : 2, d, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+            return false;
+        if (c) {
+            if (!encode(&mp.c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, batched ? 3 : 2, c, dims, str, box,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+                return false;
+        } else {
+            mp.c = mp.d;   // never read when has_c == 0
+        }
+    }
+    return true;
+}
+
+template <int BN, int STAGES, int KIND>
+dg_status launch_normal(const GemmMaps &mp, const dg::GemmParams &p, int grid, cudaStream_t st) {
+    using L = dg::NormalLayout<BN, STAGES>;
+    auto kern = dg::gemm_normal_kernel<BN, STAGES, KIND>;
+    static std::atomic<uint64_t> attr_done[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev].load()) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) != cudaSuccess)
+            return DG_ERR_CUDA;
+        attr_done[dev].store(1);
+    }
+    kern<<<grid, dg::GEMM_THREADS, L::ALLOC, st>>>(mp.a, mp.b, mp.sfa, mp.c, mp.d, p);
+    return from_cuda(cudaGetLastError());
+}
+
+// Tile width: 256 columns unless N is small; the persistent grid covers all SMs or all tiles.
+template <int KIND>
+dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
+                   const int32_t *layout, const int32_t *masked_m, int rows, int N, int K, int G, cudaStream_t st) {
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    dg::GemmParams p{};
+    p.M = rows;
+    p.N = N;
+    p.K = K;
+    p.G = G;
+    p.Kb = K / 128;
+    p.Nb = (N + 127) / 128;
+    p.m_blocks = (rows + dg::BM - 1) / dg::BM;
+    p.has_c = c != nullptr;
+    p.sfb = sfb;
+    p.grouped_layout = layout;
+    p.masked_m = masked_m;
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.err = di->err;
+    p.timeout_ns = wait_limit_ns();
+    const bool batched = KIND == dg::KIND_MASKED;
+    GemmMaps mp;
+    if (N > 128) {
+        constexpr int BN = 256;
+        p.n_blocks = (N + BN - 1) / BN;
+        const int tiles = batched ? G * p.m_blocks * p.n_blocks : p.m_blocks * p.n_blocks;
+        p.num_tiles = batched ? 0 : tiles;
+        if (!build_maps<BN>(mp, a, sfa, b, c, d, rows, N, K, G, batched)) return DG_ERR_INVALID_ARG;
+        const int grid = tiles < di->sm_count ? tiles : di->sm_count;
+        return launch_normal<BN, 3, KIND>(mp, p, grid, st);
+    } else {
+        constexpr int BN = 128;
+        p.n_blocks = (N + BN - 1) / BN;
+        const int tiles = batched ? G * p.m_blocks * p.n_blocks : p.m_blocks * p.n_blocks;
+        p.num_tiles = batched ? 0 : tiles;
+        if (!build_maps<BN>(mp, a, sfa, b, c, d, rows, N, K, G, batched)) return DG_ERR_INVALID_ARG;
+        const int grid = tiles < di->sm_count ? tiles : di->sm_count;
+        return launch_normal<BN, 5, KIND>(mp, p, grid, st);
+    }
+}
+
+dg_status check_gemm_common(const void *a, const float *sfa, const void *b, const float *sfb, const void *c,
+                            const void *d, int N, int K) {
+    if (!a || !sfa || !b || !sfb || !d) return DG_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || K % 128 != 0 || N % 8 != 0) return DG_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(sfa) || !aligned16(sfb) || !aligned16(d) ||
+        (c && !aligned16(c)))
+        return DG_ERR_ALIGNMENT;
+    return DG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dg_status dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
+                         int M, int N, int K, void *stream) {
+    if (M < 0) return DG_ERR_INVALID_ARG;
+    dg_status s = check_gemm_common(a, sfa, b, sfb, c, d, N, K);
+    if (s != DG_OK) return s;
+    if (M == 0) return DG_OK;
+    return run_gemm<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, nullptr, M, N, K, 1,
+                                    static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
+                                              const void *c, void *d, const int32_t *grouped_layout, int M_sum,
+                                              int N, int K, int G, void *stream) {
+    if (M_sum < 0 || M_sum % 128 != 0 || G <= 0 || !grouped_layout) return DG_ERR_INVALID_ARG;
+    dg_status s = check_gemm_common(a, sfa, b, sfb, c, d, N, K);
+    if (s != DG_OK) return s;
+    if (M_sum == 0) return DG_OK;
+    return run_gemm<dg::KIND_CONTIGUOUS>(a, sfa, b, sfb, c, d, grouped_layout, nullptr, M_sum, N, K, G,
+                                         static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb,
+                                          const void *c, void *d, const int32_t *masked_m, int expected_m, int G,
+                                          int M_max, int N, int K, void *stream) {
+    (void)expected_m;
+    if (G <= 0 || M_max < 0 || !masked_m || expected_m < 0) return DG_ERR_INVALID_ARG;
+    dg_status s = check_gemm_common(a, sfa, b, sfb, c, d, N, K);
+    if (s != DG_OK) return s;
+    if (M_max == 0) return DG_OK;
+    return run_gemm<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, nullptr, masked_m, M_max, N, K, G,
+                                     static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_transform_sf(const float *sf_kmajor, float *sf_mnmajor, int batch, int MN, int Kb, void *stream) {
+    if (!sf_kmajor || !sf_mnmajor || batch < 0 || MN < 0 || Kb < 0 || batch > 65535) return DG_ERR_INVALID_ARG;
+    if (batch == 0 || Kb == 0) return DG_OK;
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    const int ld = pad4(MN);
+    if (ld == 0) return DG_OK;
+    dim3 grid((ld + 31) / 32, (Kb + 31) / 32, batch);
+    dg::transform_sf_kernel<<<grid, dim3(32, 8), 0, static_cast<cudaStream_t>(stream)>>>(sf_kmajor, sf_mnmajor, MN,
+                                                                                         Kb, ld);
+    return from_cuda(cudaGetLastError());
+}
+
+dg_status dg_cast_fp8_per_token(const void *x, void *q, float *sfa, int batch, int M, int K, void *stream) {
+    if (!x || !q || !sfa || batch < 0 || M < 0 || K <= 0 || K % 128 != 0 || batch > 65535) return DG_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(sfa)) return DG_ERR_ALIGNMENT;
+    if (batch == 0 || M == 0) return DG_OK;
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    const int Kb = K / 128;
+    dim3 grid((M + 31) / 32, (Kb + 3) / 4, batch);
+    if (grid.y > 65535) return DG_ERR_INVALID_ARG;
+    dg::cast_per_token_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16 *>(x), static_cast<uint8_t *>(q), sfa, M, K, pad4(M));
+    return from_cuda(cudaGetLastError());
+}
+
+dg_status dg_cast_fp8_per_block(const void *x, void *q, float *sfb, int batch, int N, int K, void *stream) {
+    if (!x || !q || !sfb || batch < 0 || N < 0 || K <= 0 || K % 128 != 0 || batch > 65535) return DG_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(sfb)) return DG_ERR_ALIGNMENT;
+    if (batch == 0 || N == 0) return DG_OK;
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    dim3 grid(K / 128, (N + 127) / 128, batch);
+    if (grid.y > 65535) return DG_ERR_INVALID_ARG;
+    dg::cast_per_block_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16 *>(x), static_cast<uint8_t *>(q), sfb, N, K);
+    return from_cuda(cudaGetLastError());
+}
+
+int dg_sf_ld(int mn) { return mn <= 0 ? 0 : pad4(mn); }
+
+dg_status dg_get_device_error(void *stream) {
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DG_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, di->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DG_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(di->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return DG_ERR_CUDA;
+    }
+    if (v == dg::ERR_TIMEOUT) return DG_ERR_TIMEOUT;
+    if (v != 0) return DG_ERR_DEVICE;
+    return DG_OK;
+}
+
+const char *dg_status_string(dg_status status) {
+    switch (status) {
+        case DG_OK: return "DG_OK";
+        case DG_ERR_INVALID_ARG: return "DG_ERR_INVALID_ARG";
+        case DG_ERR_ALIGNMENT: return "DG_ERR_ALIGNMENT";
+        case DG_ERR_UNSUPPORTED: return "DG_ERR_UNSUPPORTED";
+        case DG_ERR_CUDA: return "DG_ERR_CUDA";
+        case DG_ERR_TIMEOUT: return "DG_ERR_TIMEOUT";
+        case DG_ERR_DEVICE: return "DG_ERR_DEVICE";
+    }
+    return "DG_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,103 @@
+"""GPU parity of the dense FP8 block-scaled NT GEMM against the oracle, element by element,
+within |D - ref| <= 2^-7·|ref| + 1e-2·rms(ref). Operands come from the CUDA casts, which are
+checked bit-exact against the oracle casts first, so both sides see the same e4m3 codes and
+scales."""
+import numpy as np
+import pytest
+import torch
+
+from moe_grouped_gemm_sm_b200 import build, ops, synth
+from tests.gpu_util import assert_close, bf16_dev, bf16_host_f64, host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+def quantised(oracle, M, N, K, with_c, salt):
+    x, w, c = synth.dense_inputs(M, N, K, with_c, salt=salt)
+    a, sfa = ops.cast_per_token(bf16_dev(x))
+    b, sfb = ops.cast_per_block(bf16_dev(w))
+    ao, sfao = oracle.cast_per_token(x)
+    bo, sfbo = oracle.cast_per_block(w)
+    assert np.array_equal(host(a), ao) and np.array_equal(host(b), bo)
+    assert np.array_equal(host(sfa), sfao) and np.array_equal(host(sfb), sfbo)
+    return (a, sfa, b, sfb, bf16_dev(c) if c is not None else None), (ao, sfao, bo, sfbo, c)
+
+
+SMALL = [
+    (1, 128, 128), (63, 264, 256), (64, 128, 384), (65, 2112, 256), (127, 136, 512), (129, 520, 128),
+    (300, 384, 640), (256, 256, 1024), (200, 8, 256), (130, 1000, 896), (512, 2304, 256),
+]
+
+
+@pytest.mark.parametrize("M,N,K", SMALL)
+@pytest.mark.parametrize("with_c", [False, True])
+def test_dense_small_full_compare(oracle, M, N, K, with_c):
+    dv, hv = quantised(oracle, M, N, K, with_c, salt=M * 7 + N + K)
+    a, sfa, b, sfb, c = dv
+    d = ops.fp8_gemm_nt(a, sfa, b, sfb, c)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_nt(*hv)
+    assert_close(bf16_host_f64(d), ref, f"{M}x{N}x{K} c={with_c}")
+
+
+def test_dense_c_aliases_d(oracle):
+    M, N, K = 192, 384, 512
+    dv, hv = quantised(oracle, M, N, K, True, salt=9)
+    a, sfa, b, sfb, c = dv
+    d = c.clone()
+    ops.fp8_gemm_nt(a, sfa, b, sfb, d, out=d)
+    assert_close(bf16_host_f64(d), oracle.gemm_nt(*hv), "c aliases d")
+
+
+def test_dense_repeatable_and_deterministic(oracle):
+    M, N, K = 300, 520, 1024
+    dv, _ = quantised(oracle, M, N, K, True, salt=3)
+    d1 = ops.fp8_gemm_nt(*dv)
+    d2 = ops.fp8_gemm_nt(*dv)
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+
+
+PAGE_SHAPES = [(2112, 7168), (24576, 1536), (32768, 512), (7168, 16384), (4096, 7168), (7168, 2048)]
+
+
+def sample_rows(M, per_tile=2, extra=16, seed=0):
+    """First and last row of every 128-row tile plus seeded random rows."""
+    rows = set()
+    for t in range(0, M, 128):
+        rows.add(t)
+        rows.add(min(M, t + 128) - 1)
+    rng = np.random.default_rng(seed)
+    rows.update(rng.integers(0, M, extra).tolist())
+    return np.array(sorted(rows), np.int32)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("M", [64, 128])
+@pytest.mark.parametrize("N,K", PAGE_SHAPES)
+def test_decode_shapes_full_compare(oracle, M, N, K):
+    with_c = not (M == 64 and (N, K) == (2112, 7168))      # the 64x2112x7168 case has C = 0
+    dv, hv = quantised(oracle, M, N, K, with_c, salt=N + K + M)
+    d = ops.fp8_gemm_nt(*dv)
+    torch.cuda.synchronize()
+    rows = np.arange(M, dtype=np.int32) if N * K <= 16 * 2 ** 20 else sample_rows(M, extra=8)
+    ref = oracle.gemm_nt(*hv, rows=rows)
+    assert_close(bf16_host_f64(d)[rows], ref, f"decode {M}x{N}x{K}")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("N,K", PAGE_SHAPES)
+def test_prefill_shapes_sampled_rows(oracle, N, K):
+    M = 4096
+    dv, hv = quantised(oracle, M, N, K, True, salt=N + K)
+    d = ops.fp8_gemm_nt(*dv)
+    torch.cuda.synchronize()
+    rows = sample_rows(M, extra=16, seed=N)
+    if N * K > 64 * 2 ** 20:
+        rows = rows[::2]
+    ref = oracle.gemm_nt(*hv, rows=rows)
+    assert_close(bf16_host_f64(d)[rows], ref, f"prefill 4096x{N}x{K}")
