@@ -21,6 +21,9 @@ groups of U{2048..6144} rows padded to 128, masked MoE with masked_m ~ U{64..256
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 _GAMMA = np.uint64(0x9E3779B97F4A7C15)
@@ -32,7 +35,15 @@ BASE_SEED = 2026
 # stream offsets from the base seed
 STREAM_A, STREAM_B, STREAM_C, STREAM_GROUPS, STREAM_GARBAGE = 0, 1, 2, 3, 4
 
-_CHUNK = 1 << 24
+_CHUNK = 1 << 22
+_POOL = None
+
+
+def _pool():
+    global _POOL
+    if _POOL is None:
+        _POOL = ThreadPoolExecutor(max_workers=max(1, min(32, os.cpu_count() or 1)))
+    return _POOL
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
@@ -82,11 +93,19 @@ def normal_bf16(seed: int, shape, sigma: float = 1.0) -> np.ndarray:
     """bf16 bit patterns (uint16) of N(0, sigma^2) draws, filled in row-major order."""
     n = int(np.prod(shape))
     out = np.empty(n, dtype=np.uint16)
-    for s in range(0, n, _CHUNK):
+
+    def fill(s):
         cnt = min(_CHUNK, n - s)
         # chunks start on even draw indices so the pairing never straddles two chunks
         z = normal_f64(seed, cnt, start_pair=s // 2)
         out[s:s + cnt] = f32_to_bf16_bits((z * sigma).astype(np.float32))
+
+    starts = range(0, n, _CHUNK)
+    if n > 2 * _CHUNK:
+        list(_pool().map(fill, starts))
+    else:
+        for s in starts:
+            fill(s)
     return out.reshape(shape)
 
 
