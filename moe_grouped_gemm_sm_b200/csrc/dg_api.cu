@@ -79,6 +79,19 @@ uint64_t wait_limit_ns() {
     return v;
 }
 
+// Tile-width override for experiments (DG_FORCE_BN=128|256); 0 = heuristic.
+int forced_bn() {
+    static std::atomic<int> cached{-1};
+    int v = cached.load();
+    if (v < 0) {
+        v = 0;
+        if (const char *s = std::getenv("DG_FORCE_BN")) v = std::atoi(s);
+        if (v != 128 && v != 256) v = 0;
+        cached.store(v);
+    }
+    return v;
+}
+
 // Encodes a tiled tensor map. dims/box are innermost first; strides (bytes) for dims 1..rank-1.
 bool encode(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
             const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle sw) {
@@ -189,7 +202,8 @@ dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *
     p.timeout_ns = wait_limit_ns();
     const bool batched = KIND == dg::KIND_MASKED;
     GemmMaps mp;
-    if (N > 128) {
+    const int fbn = forced_bn();
+    if (fbn ? fbn == 256 : N > 128) {
         constexpr int BN = 256;
         p.n_blocks = (N + BN - 1) / BN;
         const int tiles = batched ? G * p.m_blocks * p.n_blocks : p.m_blocks * p.n_blocks;

@@ -68,11 +68,12 @@ struct NormalLayout {
     static constexpr int OFF_D = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_SFA = OFF_D + 8 * SLAB_BYTES;
     static constexpr int OFF_BAR = OFF_SFA + SFA_STAGES * BM * 4;
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * SFA_STAGES + 4 + 8;
+    static constexpr int NBUF = 512 / BN;               // TMEM partial buffers (MMA run-ahead)
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * SFA_STAGES + 2 * NBUF + 8;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int BYTES = OFF_MISC + static_cast<int>(sizeof(WaitCtx));
     static constexpr int ALLOC = BYTES + 1024;          // slack to align the base to 1024 B
-    static constexpr uint32_t TMEM_COLS = 2 * BN;       // two accumulator buffers
+    static constexpr uint32_t TMEM_COLS = 512;          // NBUF partial buffers of BN columns
     static_assert(OFF_B % 1024 == 0 && OFF_D % 1024 == 0, "1024-byte aligned operand tiles");
     static_assert(ALLOC <= 232448, "shared memory budget");
 };
@@ -131,19 +132,46 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams &p) {
     return ti;
 }
 
-template <int N>
-__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[N]) {
-    static_assert(N == 32, "wait barrier for 32 registers");
-    // The registers are in/out operands so that no use of them is scheduled before the wait.
-    asm volatile(
-        "tcgen05.wait::ld.sync.aligned;"
-        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-          "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-          "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
-          "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
-          "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-        :
-        : "memory");
+// tcgen05.wait::ld with the loaded registers as in/out operands, so that no use of them can
+// be scheduled before the wait.
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
+// The same for one 32-register batch.
+__device__ __forceinline__ void tmem_ld_wait_regs32(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
+                   "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
+                   "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+// The same for four 16-register groups (64 registers).
+__device__ __forceinline__ void tmem_ld_wait_regs4(uint32_t (&r)[4][16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0][0]), "+r"(r[0][1]), "+r"(r[0][2]), "+r"(r[0][3]), "+r"(r[0][4]), "+r"(r[0][5]),
+                   "+r"(r[0][6]), "+r"(r[0][7]), "+r"(r[0][8]), "+r"(r[0][9]), "+r"(r[0][10]), "+r"(r[0][11]),
+                   "+r"(r[0][12]), "+r"(r[0][13]), "+r"(r[0][14]), "+r"(r[0][15]),
+                   "+r"(r[1][0]), "+r"(r[1][1]), "+r"(r[1][2]), "+r"(r[1][3]), "+r"(r[1][4]), "+r"(r[1][5]),
+                   "+r"(r[1][6]), "+r"(r[1][7]), "+r"(r[1][8]), "+r"(r[1][9]), "+r"(r[1][10]), "+r"(r[1][11]),
+                   "+r"(r[1][12]), "+r"(r[1][13]), "+r"(r[1][14]), "+r"(r[1][15]),
+                   "+r"(r[2][0]), "+r"(r[2][1]), "+r"(r[2][2]), "+r"(r[2][3]), "+r"(r[2][4]), "+r"(r[2][5]),
+                   "+r"(r[2][6]), "+r"(r[2][7]), "+r"(r[2][8]), "+r"(r[2][9]), "+r"(r[2][10]), "+r"(r[2][11]),
+                   "+r"(r[2][12]), "+r"(r[2][13]), "+r"(r[2][14]), "+r"(r[2][15]),
+                   "+r"(r[3][0]), "+r"(r[3][1]), "+r"(r[3][2]), "+r"(r[3][3]), "+r"(r[3][4]), "+r"(r[3][5]),
+                   "+r"(r[3][6]), "+r"(r[3][7]), "+r"(r[3][8]), "+r"(r[3][9]), "+r"(r[3][10]), "+r"(r[3][11]),
+                   "+r"(r[3][12]), "+r"(r[3][13]), "+r"(r[3][14]), "+r"(r[3][15])
+                 :
+                 : "memory");
 }
 
 template <int BN, int STAGES, int KIND>
@@ -163,10 +191,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint64_t *sfa_full = empty + STAGES;
     uint64_t *sfa_empty = sfa_full + SFS;
     uint64_t *tfull = sfa_empty + SFS;
-    uint64_t *tempty = tfull + 2;
-    uint64_t *cfull = tempty + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_MISC + 4);
+    uint64_t *tempty = tfull + L::NBUF;
+    uint64_t *cfull = tempty + L::NBUF;
+    WaitCtx *ctx = reinterpret_cast<WaitCtx *>(smem + L::OFF_MISC);
+    volatile int *abort_flag = &ctx->abort;
     const float *sfa_ring = reinterpret_cast<const float *>(smem + L::OFF_SFA);
 
     const int warp = threadIdx.x >> 5;
@@ -181,12 +209,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             mbar_init(&sfa_full[j], 1);
             mbar_init(&sfa_empty[j], 8);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < L::NBUF; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 8);
         }
         for (int w = 0; w < 8; ++w) mbar_init(&cfull[w], 1);
-        *abort_flag = 0;
+        ctx->abort = 0;
+        ctx->err = p.err;
+        ctx->limit_ns = p.timeout_ns;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -197,13 +227,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tma_prefetch_desc(&tm_d);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, L::TMEM_COLS);
+        tmem_alloc(&ctx->tmem_base, L::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_base = ctx->tmem_base;
 
     const int num_tiles = (KIND == KIND_MASKED) ? masked_num_tiles(p) : p.num_tiles;
     if (KIND == KIND_MASKED && blockIdx.x == 0 && threadIdx.x == 0) {
@@ -212,7 +242,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
 
     if (warp < 4) {
-        reg_dealloc<88>();
+        reg_dealloc<56>();
         if (warp == 0 && lane == 0) {
             // ---------------- TMA producer ----------------
             uint32_t it = 0;
@@ -225,10 +255,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 for (int kb = 0; kb < p.Kb; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err, p.timeout_ns)) break;
+                    if (!mbar_wait(&empty[s], ph ^ 1, ctx)) break;
                     const int j = it % SFS;
                     const uint32_t phj = (it / SFS) & 1;
-                    if (!mbar_wait(&sfa_empty[j], phj ^ 1, abort_flag, p.err, p.timeout_ns)) break;
+                    if (!mbar_wait(&sfa_empty[j], phj ^ 1, ctx)) break;
                     mbar_arrive_expect_tx(&full[s], L::A_BYTES + L::B_BYTES);
                     uint8_t *sa = smem + L::OFF_A + s * L::A_BYTES;
                     uint8_t *sb = smem + L::OFF_B + s * L::B_BYTES;
@@ -255,10 +285,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 for (int kb = 0; kb < p.Kb; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    const int b = it & 1;
-                    const uint32_t phb = (it >> 1) & 1;
-                    if (!mbar_wait(&full[s], ph, abort_flag, p.err, p.timeout_ns)) break;
-                    if (!mbar_wait(&tempty[b], phb ^ 1, abort_flag, p.err, p.timeout_ns)) break;
+                    const int b = it % L::NBUF;
+                    const uint32_t phb = (it / L::NBUF) & 1;
+                    if (!mbar_wait(&full[s], ph, ctx)) break;
+                    if (!mbar_wait(&tempty[b], phb ^ 1, ctx)) break;
                     tc_fence_after();
                     const uint64_t ad = sdesc_k_sw128(smem_u32(smem + L::OFF_A + s * L::A_BYTES));
                     const uint64_t bd = sdesc_k_sw128(smem_u32(smem + L::OFF_B + s * L::B_BYTES));
@@ -272,7 +302,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             }
         }
     } else {
-        reg_alloc<208>();
+        reg_alloc<224>();
         // ---------------- math warpgroups: promotion + epilogue ----------------
         const int mw = warp - 4;               // 0..7
         const int wg = mw >> 2;                // column half
@@ -299,44 +329,59 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         tma_load_2d(&tm_c, &cfull[mw], slab + bx * 4096, col0 + bx * 64, row0);
                 }
             }
-            float acc[HALF];
+            float2 acc[HALF / 2];
 #pragma unroll
-            for (int i = 0; i < HALF; ++i) acc[i] = 0.f;
-            float sb = __ldg(sfb_row);
+            for (int i = 0; i < HALF / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+            // sfb of this warp's n-block for 32 consecutive K blocks, one per lane; the next
+            // window is fetched a full window ahead and broadcast by shuffle
+            float sb_win = lane < p.Kb ? __ldg(sfb_row + lane) : 0.f;
+            float sb_nxt = 32 + lane < p.Kb ? __ldg(sfb_row + 32 + lane) : 0.f;
             for (int kb = 0; kb < p.Kb; ++kb, ++it) {
-                const int b = it & 1;
-                const uint32_t phb = (it >> 1) & 1;
+                const int b = it % L::NBUF;
+                const uint32_t phb = (it / L::NBUF) & 1;
                 const int j = it % SFS;
                 const uint32_t phj = (it / SFS) & 1;
-                const float sb_next = (kb + 1 < p.Kb) ? __ldg(sfb_row + kb + 1) : 0.f;
+                if ((kb & 31) == 0 && kb > 0) {
+                    sb_win = sb_nxt;
+                    sb_nxt = kb + 32 + lane < p.Kb ? __ldg(sfb_row + kb + 32 + lane) : 0.f;
+                }
+                const float sb = __shfl_sync(0xFFFFFFFFu, sb_win, kb & 31);
                 // every lane waits; the outcome is made warp-uniform before any .sync.aligned op
-                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sfa_full[j], phj, abort_flag, p.err, p.timeout_ns));
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sfa_full[j], phj, ctx));
                 if (!ok) break;
                 const float sa = sfa_ring[j * BM + q * 32 + lane];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sfa_empty[j]);
-                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], phb, abort_flag, p.err, p.timeout_ns));
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], phb, ctx));
                 if (!ok) break;
                 tc_fence_after();
                 const float scale = sa * sb;
+                const float2 scale2 = make_float2(scale, scale);
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                        static_cast<uint32_t>(b * BN + wg * HALF);
+                // 32-column batches, double-buffered in registers: the TMEM load of batch c+1 is
+                // in flight while batch c is folded into the accumulator (tcgen05.wait::ld waits
+                // for every outstanding load, so at most one batch is in flight)
+                uint32_t r[2][32];
+                tmem_ld32(taddr, r[0]);
+                tmem_ld_wait_regs32(r[0]);
 #pragma unroll
                 for (int c = 0; c < HALF / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(taddr + c * 32, r);
-                    tmem_ld_wait_regs(r);
+                    if (c + 1 < HALF / 32) tmem_ld32(taddr + (c + 1) * 32, r[(c + 1) & 1]);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(__uint_as_float(r[i]), scale, acc[c * 32 + i]);
+                    for (int i = 0; i < 16; ++i)
+                        acc[c * 16 + i] = __ffma2_rn(make_float2(__uint_as_float(r[c & 1][2 * i]),
+                                                                 __uint_as_float(r[c & 1][2 * i + 1])),
+                                                     scale2, acc[c * 16 + i]);
+                    if (c + 1 < HALF / 32) tmem_ld_wait_regs32(r[(c + 1) & 1]);
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[b]);
-                sb = sb_next;
             }
             if (!ok) break;
             if (p.has_c) {
-                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&cfull[mw], ctile & 1, abort_flag, p.err, p.timeout_ns));
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&cfull[mw], ctile & 1, ctx));
                 if (!ok) break;
                 ++ctile;
             } else {
@@ -352,7 +397,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     uint4 *pchunk = reinterpret_cast<uint4 *>(slab + bx * 4096 + lane * 128 + ((ch ^ (lane & 7)) * 16));
                     float v[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = acc[bx * 64 + ch * 8 + e];
+                    for (int e = 0; e < 4; ++e) {
+                        v[2 * e] = acc[bx * 32 + ch * 4 + e].x;
+                        v[2 * e + 1] = acc[bx * 32 + ch * 4 + e].y;
+                    }
                     if (p.has_c) {
                         const uint4 cv = *pchunk;
                         const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};

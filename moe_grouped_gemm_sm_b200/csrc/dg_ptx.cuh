@@ -58,22 +58,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits until the phase with the given parity has completed. Gives up after `limit_ns`
-// (measured on %globaltimer) or as soon as *abort is set by another warp; on a timeout it
-// records ERR_TIMEOUT in the device error word and raises *abort so that every role of the
-// CTA leaves its loop. Returns false when it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int *err, uint64_t limit_ns) {
+// Shared-memory context of the bounded waits: kept in shared memory so that the waits' slow
+// path does not hold the error pointer and the time limit in registers across the hot loops.
+struct WaitCtx {
+    uint32_t tmem_base;   // TMEM address written by tcgen05.alloc
+    int abort;            // raised by the first wait that times out; every role then leaves
+    int *err;             // device error word
+    uint64_t limit_ns;    // per-wait limit on %globaltimer
+};
+
+// Waits until the phase with the given parity has completed. Gives up after ctx->limit_ns or as
+// soon as ctx->abort is raised by another warp; on a timeout it records ERR_TIMEOUT in the
+// device error word and raises ctx->abort so that every role of the CTA leaves its loop.
+// Returns false when it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitCtx *ctx) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
+    volatile int *abort = &ctx->abort;
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(a, parity)) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > limit_ns) {
-            report_error(err, ERR_TIMEOUT);
+        if (globaltimer_ns() - t0 > ctx->limit_ns) {
+            report_error(ctx->err, ERR_TIMEOUT);
             *abort = 1;
             return false;
         }
