@@ -92,6 +92,18 @@ int forced_bn() {
     return v;
 }
 
+// CTA-pair override for experiments (DG_FORCE_PAIR=0|1); -1 = heuristic.
+int forced_pair() {
+    static std::atomic<int> cached{-2};
+    int v = cached.load();
+    if (v == -2) {
+        v = -1;
+        if (const char *s = std::getenv("DG_FORCE_PAIR")) v = std::atoi(s) ? 1 : 0;
+        cached.store(v);
+    }
+    return v;
+}
+
 // Encodes a tiled tensor map. dims/box are innermost first; strides (bytes) for dims 1..rank-1.
 bool encode(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
             const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle sw) {
@@ -113,14 +125,20 @@ struct GemmMaps {
     CUtensorMap a, b, sfa, c, d;
 };
 
-// Operand maps of one GEMM call. rows = rows of A/C/D per group; batched = 3D maps over G
-// groups for A, sfa, C and D (masked layout).
-template <int BN>
-bool build_maps(GemmMaps &mp, const void *a, const float *sfa, const void *b, const void *c, void *d,
-                int rows, int N, int K, int G, bool batched) {
-    const uint64_t Kb = static_cast<uint64_t>(K / 128);
-    const uint64_t ld = static_cast<uint64_t>(pad4(rows));
+// Operand maps of one GEMM call. rows = rows of A/C/D per group; b_rows = rows of B one CTA
+// loads; batched = 3D maps over G groups for A, C and D (masked layout).
+bool build_maps(GemmMaps &mp, const void *a, const float *sfa, const void *b, const void *c, void *d, int rows, int N,
+                int K, int G, int b_rows, bool batched) {
     const uint64_t Gg = static_cast<uint64_t>(G);
+    {   // sfa: fp32 [G?][Kb][pad4(rows)], box 128 x 1 (one K block's scales of a 128-row block)
+        const uint64_t Kb = static_cast<uint64_t>(K / 128), ld = static_cast<uint64_t>(pad4(rows));
+        const uint64_t dims[3] = {ld, Kb, Gg};
+        const uint64_t str[2] = {ld * 4, ld * 4 * Kb};
+        const uint32_t box[3] = {128, 1, 1};
+        if (!encode(&mp.sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, batched ? 3 : 2, sfa, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+            return false;
+    }
     {   // A: e4m3 [G?][rows][K], box 128 x 128, 128-byte swizzle
         const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows), Gg};
         const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(K) * rows};
@@ -129,19 +147,11 @@ bool build_maps(GemmMaps &mp, const void *a, const float *sfa, const void *b, co
                     CU_TENSOR_MAP_SWIZZLE_128B))
             return false;
     }
-    {   // B: e4m3 [G][N][K], box 128 x BN x 1
+    {   // B: e4m3 [G][N][K], box 128 x b_rows x 1
         const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), Gg};
         const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(K) * N};
-        const uint32_t box[3] = {128, BN, 1};
+        const uint32_t box[3] = {128, static_cast<uint32_t>(b_rows), 1};
         if (!encode(&mp.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return false;
-    }
-    {   // sfa: fp32 [G?][Kb][pad4(rows)], box 128 x 1
-        const uint64_t dims[3] = {ld, Kb, Gg};
-        const uint64_t str[2] = {ld * 4, ld * 4 * Kb};
-        const uint32_t box[3] = {128, 1, 1};
-        if (!encode(&mp.sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, batched ? 3 : 2, sfa, dims, str, box,
-                    CU_TENSOR_MAP_SWIZZLE_NONE))
             return false;
     }
     {   // C, D: bf16 [G?][rows][N], box 64 x 32, 128-byte swizzle (one box row = 128 bytes)
@@ -162,23 +172,60 @@ bool build_maps(GemmMaps &mp, const void *a, const float *sfa, const void *b, co
     return true;
 }
 
-template <int BN, int STAGES, int KIND>
-dg_status launch_normal(const GemmMaps &mp, const dg::GemmParams &p, int grid, cudaStream_t st) {
-    using L = dg::NormalLayout<BN, STAGES>;
-    auto kern = dg::gemm_normal_kernel<BN, STAGES, KIND>;
-    static std::atomic<uint64_t> attr_done[kMaxDevices];
+// Per (kernel, device): dynamic shared memory opt-in and, for CTA pairs, how many two-CTA
+// clusters can be resident at once (the persistent grid never exceeds it).
+struct KernelInfo {
+    std::atomic<int> ready{0};
+    int max_clusters = 0;
+};
+
+template <int BN, int STAGES, int KIND, bool PAIR>
+dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p, int tiles, const DeviceInfo *di, cudaStream_t st) {
+    constexpr bool PAIR_LIST = PAIR && KIND == dg::KIND_CONTIGUOUS;
+    using L = dg::GemmLayout<BN, STAGES, PAIR, PAIR_LIST>;
+    auto kern = dg::gemm_kernel<BN, STAGES, KIND, PAIR>;
+    static KernelInfo info[kMaxDevices];
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (!attr_done[dev].load()) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) != cudaSuccess)
-            return DG_ERR_CUDA;
-        attr_done[dev].store(1);
+    if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(dg::GEMM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = L::ALLOC;
+    cfg.stream = st;
+    if (PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
     }
-    kern<<<grid, dg::GEMM_THREADS, L::ALLOC, st>>>(mp.a, mp.b, mp.sfa, mp.c, mp.d, p);
-    return from_cuda(cudaGetLastError());
+    KernelInfo &ki = info[dev];
+    if (!ki.ready.load()) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!ki.ready.load()) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) != cudaSuccess)
+                return DG_ERR_CUDA;
+            if (PAIR) {
+                cfg.gridDim = dim3(2 * (di->sm_count / 2), 1, 1);
+                int n = 0;
+                if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return DG_ERR_CUDA;
+                ki.max_clusters = n;
+            }
+            ki.ready.store(1);
+        }
+    }
+    const int units = PAIR ? ki.max_clusters : di->sm_count;
+    const int n_units = tiles < units ? tiles : units;
+    if (n_units <= 0) return DG_OK;
+    cfg.gridDim = dim3(PAIR ? 2 * n_units : n_units, 1, 1);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mp.a, mp.b, mp.sfa, mp.c, mp.d, p);
+    return from_cuda(e);
 }
 
-// Tile width: 256 columns unless N is small; the persistent grid covers all SMs or all tiles.
+// Tile-shape choice. Pairs of CTAs (256-row tiles, cta_group::2) for every layout with more
+// than 128 rows per group; single CTAs (128-row tiles) otherwise. 256 columns per tile unless
+// N <= 128. Stages fill the shared-memory budget.
 template <int KIND>
 dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
                    const int32_t *layout, const int32_t *masked_m, int rows, int N, int K, int G, cudaStream_t st) {
@@ -192,8 +239,9 @@ dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *
     p.G = G;
     p.Kb = K / 128;
     p.Nb = (N + 127) / 128;
-    p.m_blocks = (rows + dg::BM - 1) / dg::BM;
+    p.ld_sfa = pad4(rows);
     p.has_c = c != nullptr;
+    p.sfa = sfa;
     p.sfb = sfb;
     p.grouped_layout = layout;
     p.masked_m = masked_m;
@@ -201,25 +249,31 @@ dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *
     p.err = di->err;
     p.timeout_ns = wait_limit_ns();
     const bool batched = KIND == dg::KIND_MASKED;
-    GemmMaps mp;
     const int fbn = forced_bn();
-    if (fbn ? fbn == 256 : N > 128) {
-        constexpr int BN = 256;
-        p.n_blocks = (N + BN - 1) / BN;
-        const int tiles = batched ? G * p.m_blocks * p.n_blocks : p.m_blocks * p.n_blocks;
-        p.num_tiles = batched ? 0 : tiles;
-        if (!build_maps<BN>(mp, a, sfa, b, c, d, rows, N, K, G, batched)) return DG_ERR_INVALID_ARG;
-        const int grid = tiles < di->sm_count ? tiles : di->sm_count;
-        return launch_normal<BN, 3, KIND>(mp, p, grid, st);
+    const int bn = fbn ? fbn : (N > 128 ? 256 : 128);
+    const int fpair = forced_pair();
+    bool pair = fpair >= 0 ? fpair == 1 : rows > 128;
+    if (KIND == dg::KIND_CONTIGUOUS && rows / 128 > dg::MAX_PAIR_BLOCKS) pair = false;
+    if (bn != 256) pair = false;                       // pairs are built for 256-column tiles
+    GemmMaps mp;
+    const int m_units = (rows + (pair ? 255 : 127)) / (pair ? 256 : 128);
+    p.n_blocks = (N + bn - 1) / bn;
+    int tiles;
+    if (KIND == dg::KIND_MASKED) {
+        tiles = G * m_units * p.n_blocks;                 // upper bound; the kernel reads masked_m
+    } else if (KIND == dg::KIND_CONTIGUOUS && pair) {
+        tiles = (rows / 128 / 2 + G) * p.n_blocks;        // upper bound on expert-local pairs
     } else {
-        constexpr int BN = 128;
-        p.n_blocks = (N + BN - 1) / BN;
-        const int tiles = batched ? G * p.m_blocks * p.n_blocks : p.m_blocks * p.n_blocks;
-        p.num_tiles = batched ? 0 : tiles;
-        if (!build_maps<BN>(mp, a, sfa, b, c, d, rows, N, K, G, batched)) return DG_ERR_INVALID_ARG;
-        const int grid = tiles < di->sm_count ? tiles : di->sm_count;
-        return launch_normal<BN, 5, KIND>(mp, p, grid, st);
+        tiles = m_units * p.n_blocks;
     }
+    p.num_tiles = (KIND == dg::KIND_MASKED || (KIND == dg::KIND_CONTIGUOUS && pair)) ? 0 : tiles;
+    const int b_rows = pair ? bn / 2 : bn;
+    if (!build_maps(mp, a, sfa, b, c, d, rows, N, K, G, b_rows, batched)) return DG_ERR_INVALID_ARG;
+    if (pair) {
+        return launch_gemm<256, 4, KIND, true>(mp, p, tiles, di, st);
+    }
+    if (bn == 256) return launch_gemm<256, 3, KIND, false>(mp, p, tiles, di, st);
+    return launch_gemm<128, 5, KIND, false>(mp, p, tiles, di, st);
 }
 
 dg_status check_gemm_common(const void *a, const float *sfa, const void *b, const float *sfb, const void *c,
