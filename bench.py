@@ -1,21 +1,27 @@
 #!/usr/bin/env python
 """Benchmark of the FP8 block-scaled NT GEMM hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference] [--workload prefill|decode64|decode128]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+                    [--workload prefill|decode64|decode128|contiguous|masked] [--only N,K]
 
-One step = one pass of the hot path over the workload: for each (N, K) shape of the workload,
-the per-token FP8 cast of the bf16 activations A [M,K] (1x128 scales, MN-major layout) and the
-GEMM D = C + A·Bᵀ with 128x128-block-scaled e4m3 weights. The weights are cast once, before the
-timed region (offline, as in inference); that cast is timed on its own and reported under
-"weight_cast". Inputs are the seeded synthetic recipe of moe_grouped_gemm_sm_b200.synth:
-A, B ~ N(0,1) and C ~ N(0,0.1) in bf16.
+One step = one pass of the hot path over the workload: for each problem of the workload, the
+per-token FP8 cast of its bf16 activations (1x128 scales written in the MN-major layout) and
+the GEMM D = C + A·Bᵀ with 128x128-block-scaled e4m3 weights (dense, M-grouped contiguous or
+M-grouped masked). Weights are cast once, before the timed region (offline, as in inference);
+that cast is timed on its own and reported under "weight_cast". Inputs follow the seeded
+synthetic recipe of moe_grouped_gemm_sm_b200.synth: A, B ~ N(0,1) and C ~ N(0,0.1) in bf16;
+contiguous experts hold U{2048..6144} rows padded to 128; masked experts U{64..256} rows.
+
+The default workload (the one the headline number is quoted on) is the dense prefill set:
+M = 4096 with (N,K) in the six DeepSeek-V3 GEMM shapes and a C addend.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a device synchronise,
-timed with CUDA events on the launching stream; the max over ranks is reported. The working set
-of one step (activations, weights, C and D of six shapes) is far larger than the 126 MB L2, so
-no explicit flush is needed between steps. Per-kernel durations come from CUDA events recorded
-around every launch inside the timed region. SM clocks and throttle reasons are sampled through
-NVML during the timed region.
+timed with CUDA events on the launching stream; the max over ranks is reported. When one step's
+working set is below 512 MB (the decode workloads), a 256 MB L2-flushing write runs at the
+start of every step, outside the per-kernel event pairs; otherwise the working set alone is far
+above the 126 MB L2. Per-kernel durations come from CUDA events recorded around every launch
+inside the timed region. SM clocks and throttle reasons are sampled through NVML during the
+timed region.
 
 Multi-GPU: the path has no exchange step, so N GPUs run N independent replicas (one process per
 GPU under torchrun), each on the full workload ("scaling": "weak"); value = all ranks' FLOPs
@@ -39,13 +45,20 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 PREFILL_SHAPES = [(2112, 7168), (24576, 1536), (32768, 512), (7168, 16384), (4096, 7168), (7168, 2048)]
+GROUPED_SHAPES = [(4096, 7168), (7168, 2048)]
 WORKLOADS = {
-    "prefill": dict(M=4096, shapes=PREFILL_SHAPES, with_c=True,
+    "prefill": dict(kind="dense", M=4096, shapes=PREFILL_SHAPES, with_c=True,
                     desc="dense FP8 NT GEMM, M=4096, (N,K) in the six DeepSeek-V3 prefill shapes, C bf16"),
-    "decode64": dict(M=64, shapes=PREFILL_SHAPES, with_c=True,
+    "decode64": dict(kind="dense", M=64, shapes=PREFILL_SHAPES, with_c=True,
                      desc="dense FP8 NT GEMM, M=64 decode, six (N,K) shapes, C bf16"),
-    "decode128": dict(M=128, shapes=PREFILL_SHAPES, with_c=True,
+    "decode128": dict(kind="dense", M=128, shapes=PREFILL_SHAPES, with_c=True,
                       desc="dense FP8 NT GEMM, M=128 decode, six (N,K) shapes, C bf16"),
+    "contiguous": dict(kind="contiguous", G=8, shapes=GROUPED_SHAPES, with_c=False,
+                       desc="M-grouped contiguous FP8 GEMM, G=8, m_g ~ U{2048..6144} padded to 128, "
+                            "(N,K) in {(4096,7168),(7168,2048)}"),
+    "masked": dict(kind="masked", G=16, M_max=256, expected_m=192, shapes=GROUPED_SHAPES, with_c=False,
+                   desc="M-grouped masked FP8 GEMM, G=16, M_max=256, masked_m ~ U{64..256}, expected_m=192, "
+                        "(N,K) in {(4096,7168),(7168,2048)}"),
 }
 METRIC = "FP8 block-scaled GEMM TFLOPS on 1×B200; % of FP8 peak / HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -168,27 +181,52 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------------
-# workload
+# workload: problems with their host inputs, FLOPs and algorithmic bytes
 # ------------------------------------------------------------------------------------------------
 
-def algorithmic_bytes(M, N, K, with_c):
-    """HBM bytes one GEMM launch must move at minimum: e4m3 A and B, fp32 scales, C and D."""
-    kb, nb = K // 128, (N + 127) // 128
-    return M * K + N * K + 4 * (M * kb + nb * kb) + 2 * M * N + (2 * M * N if with_c else 0)
-
-
-def cast_bytes(M, K):
-    """Per-token cast: 2 B read and 1 B written per element, one fp32 scale per 128 elements."""
-    return 3 * M * K + 4 * M * (K // 128)
-
-
-def make_inputs(wl):
+def make_problems(wl):
+    """Host-side problems of a workload (bf16 bit patterns from the seeded generator)."""
     from moe_grouped_gemm_sm_b200 import synth
-    out = []
+    probs = []
     for i, (N, K) in enumerate(wl["shapes"]):
-        x, w, c = synth.dense_inputs(wl["M"], N, K, wl["with_c"], salt=100 + i)
-        out.append((N, K, x, w, c))
-    return out
+        kind = wl["kind"]
+        p = dict(kind=kind, N=N, K=K, with_c=wl["with_c"], salt=100 + i)
+        if kind == "dense":
+            x, w, c = synth.dense_inputs(wl["M"], N, K, wl["with_c"], salt=100 + i)
+            p.update(rows=wl["M"], G=1, x=x, w=w, c=c, valid_rows=wl["M"])
+        elif kind == "contiguous":
+            m, layout, x, w = synth.contiguous_inputs(wl["G"], N, K, salt=100 + i)
+            p.update(rows=layout.shape[0], G=wl["G"], x=x, w=w, c=None, layout=layout, valid_rows=int(m.sum()))
+        else:
+            mm, x, w = synth.masked_inputs(wl["G"], wl["M_max"], N, K, salt=100 + i)
+            p.update(rows=wl["M_max"], G=wl["G"], x=x, w=w, c=None, masked_m=mm, valid_rows=int(mm.sum()),
+                     expected_m=wl["expected_m"])
+        p["flops"] = 2.0 * p["valid_rows"] * N * K
+        p["bytes"] = algorithmic_bytes(p)
+        probs.append(p)
+    return probs
+
+
+def algorithmic_bytes(p):
+    """HBM bytes one GEMM launch must move at minimum: the e4m3 A rows it must read, all
+    weights, fp32 scales, the D rows it must write (and C), the grouped layout or masked_m."""
+    N, K, G = p["N"], p["K"], p["G"]
+    kb, nb = K // 128, (N + 127) // 128
+    w = G * N * K + 4 * G * nb * kb
+    if p["kind"] == "dense":
+        M = p["rows"]
+        return M * K + 4 * M * kb + w + 2 * M * N * (2 if p["with_c"] else 1)
+    if p["kind"] == "contiguous":
+        M = p["rows"]                                 # the padded layout is read and written whole
+        return M * K + 4 * M * kb + w + 2 * M * N + 4 * M
+    V = p["valid_rows"]                               # masked: only rows below masked_m matter
+    return V * K + 4 * V * kb + w + 2 * V * N + 4 * G
+
+
+def cast_bytes(p):
+    """Per-token cast of all activation rows: 2 B read and 1 B written per element, plus scales."""
+    rows = p["rows"] * (p["G"] if p["kind"] == "masked" else 1)
+    return 3 * rows * p["K"] + 4 * rows * (p["K"] // 128)
 
 
 # ------------------------------------------------------------------------------------------------
@@ -208,63 +246,84 @@ def run_cuda(args):
     if world > 1:
         dist_init("nccl")
     _build.build()
-    _lib.load()
+    L = _lib.load()
     wl = WORKLOADS[args.workload]
-    M, with_c = wl["M"], wl["with_c"]
     stream = torch.cuda.current_stream(device)
     sptr = stream.cuda_stream
 
-    def to_dev(bits):
+    def bf16(bits):
         return torch.from_numpy(np.ascontiguousarray(bits, np.uint16).view(np.int16)).view(torch.bfloat16).to(device)
 
-    host = make_inputs(wl)
-    problems = []
+    probs = make_problems(wl)
     wc_ms = []
-    for (N, K, x, w, c) in host:
-        w_dev = to_dev(w)
+    for p in probs:
+        w_dev = bf16(p["w"])
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ops.cast_per_block(w_dev)                             # warm the weight cast once
         e0.record(stream)
-        b, sfb = ops.cast_per_block(w_dev)
+        p["b"], p["sfb"] = ops.cast_per_block(w_dev)
         e1.record(stream)
         torch.cuda.synchronize(device)
-        wc_ms.append((e0.elapsed_time(e1), 3 * N * K + 4 * ((N + 127) // 128) * (K // 128)))
+        nb, kb = (p["N"] + 127) // 128, p["K"] // 128
+        wc_ms.append((e0.elapsed_time(e1), p["G"] * (3 * p["N"] * p["K"] + 4 * nb * kb)))
         del w_dev
-        a_bf16 = to_dev(x)
-        cc = to_dev(c) if c is not None else None
-        a_q = torch.empty((M, K), dtype=torch.uint8, device=device)
-        sfa = torch.empty((K // 128, (M + 3) // 4 * 4), dtype=torch.float32, device=device)
-        d = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-        problems.append(dict(N=N, K=K, a=a_bf16, c=cc, aq=a_q, sfa=sfa, b=b, sfb=sfb, d=d))
+        p["a"] = bf16(p["x"])
+        p["cd"] = bf16(p["c"]) if p["c"] is not None else None
+        batch = p["G"] if p["kind"] == "masked" else 1
+        p["batch"] = batch
+        p["aq"] = torch.empty(p["a"].shape, dtype=torch.uint8, device=device)
+        p["sfa"] = torch.empty((batch, p["K"] // 128, (p["rows"] + 3) // 4 * 4), dtype=torch.float32, device=device)
+        dshape = (p["G"], p["rows"], p["N"]) if p["kind"] == "masked" else (p["rows"], p["N"])
+        p["d"] = torch.zeros(dshape, dtype=torch.bfloat16, device=device)
+        if p["kind"] == "contiguous":
+            p["gl"] = torch.from_numpy(p["layout"]).to(device)
+        if p["kind"] == "masked":
+            p["mm"] = torch.from_numpy(p["masked_m"]).to(device)
     torch.cuda.synchronize(device)
 
-    L = _lib.load()
+    def ptr(t):
+        return t.data_ptr() if t is not None else None
 
     def launch_cast(p):
-        rc = L.dg_cast_fp8_per_token(p["a"].data_ptr(), p["aq"].data_ptr(), p["sfa"].data_ptr(), 1, M, p["K"], sptr)
+        rc = L.dg_cast_fp8_per_token(ptr(p["a"]), ptr(p["aq"]), ptr(p["sfa"]), p["batch"], p["rows"], p["K"], sptr)
         if rc:
             raise _lib.DgError("dg_cast_fp8_per_token", rc)
 
     def launch_gemm(p):
-        rc = L.dg_fp8_gemm_nt(p["aq"].data_ptr(), p["sfa"].data_ptr(), p["b"].data_ptr(), p["sfb"].data_ptr(),
-                              p["c"].data_ptr() if p["c"] is not None else None, p["d"].data_ptr(), M, p["N"],
-                              p["K"], sptr)
+        if p["kind"] == "dense":
+            rc = L.dg_fp8_gemm_nt(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]), ptr(p["cd"]), ptr(p["d"]),
+                                  p["rows"], p["N"], p["K"], sptr)
+        elif p["kind"] == "contiguous":
+            rc = L.dg_m_grouped_fp8_gemm_nt_contiguous(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]),
+                                                       ptr(p["cd"]), ptr(p["d"]), ptr(p["gl"]), p["rows"], p["N"],
+                                                       p["K"], p["G"], sptr)
+        else:
+            rc = L.dg_m_grouped_fp8_gemm_nt_masked(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]),
+                                                   ptr(p["cd"]), ptr(p["d"]), ptr(p["mm"]), p["expected_m"], p["G"],
+                                                   p["rows"], p["N"], p["K"], sptr)
         if rc:
-            raise _lib.DgError("dg_fp8_gemm_nt", rc)
+            raise _lib.DgError("gemm", rc)
 
-    def step(evs=None):
-        for i, p in enumerate(problems):
-            if evs is not None:
-                evs[2 * i].record(stream)
+    # small working sets (decode) fit in L2: flush it at the start of every step
+    step_bytes = sum(p["bytes"] + cast_bytes(p) for p in probs)
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=device) if step_bytes < 512 * 2 ** 20 else None
+
+    def step(ev=None):
+        if flush is not None:
+            flush.fill_(1)
+        cur = torch.cuda.current_stream(device)
+        for i, p in enumerate(probs):
+            if ev is not None:
+                ev[3 * i].record(cur)
             launch_cast(p)
-            if evs is not None:
-                evs[2 * i + 1].record(stream)
+            if ev is not None:
+                ev[3 * i + 1].record(cur)
             launch_gemm(p)
-        if evs is not None:
-            evs[2 * len(problems)].record(stream)
+            if ev is not None:
+                ev[3 * i + 2].record(cur)
 
-    flops_step = sum(2.0 * M * p["N"] * p["K"] for p in problems)
-    launches_per_step = 2 * len(problems)
+    flops_step = sum(p["flops"] for p in probs)
+    launches_per_step = 2 * len(probs) + (1 if flush is not None else 0)
 
     for _ in range(args.warmup):
         step()
@@ -272,51 +331,78 @@ def run_cuda(args):
     if _lib.dg_get_device_error(sptr) != 0:
         raise RuntimeError("device error word set during warm-up")
 
-    nev = 2 * len(problems) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    # The timed steps replay CUDA graphs (launch-bound decode steps would otherwise measure the
+    # host): `g_step` holds one step; `g_ev` the same step with an event pair around every
+    # launch, replayed separately for the per-kernel durations.
+    cap = torch.cuda.Stream(device)
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3 * len(probs))]
+    g_step, g_ev = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        sptr = cap.cuda_stream
+        step()                                            # warm the capture stream
+        torch.cuda.synchronize(device)
+        with torch.cuda.graph(g_step, stream=cap):
+            step()
+        with torch.cuda.graph(g_ev, stream=cap):
+            step(evs)
+    sptr = stream.cuda_stream
+    torch.cuda.synchronize(device)
+    for _ in range(args.warmup):
+        g_step.replay()
+    torch.cuda.synchronize(device)
+
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(device)
     torch.cuda.synchronize(device)
     with ClockSampler(local_rank) as clk:
         start.record(stream)
         for s in range(args.steps):
-            step(evs[s])
+            g_step.replay()
         end.record(stream)
         torch.cuda.synchronize(device)
     barrier(device)
     local_ms = start.elapsed_time(end) / args.steps
     if _lib.dg_get_device_error(sptr) != 0:
         raise RuntimeError("device error word set during the timed region")
-
-    # per-kernel averages over the timed steps
-    cast_ms = [statistics.fmean(evs[s][2 * i].elapsed_time(evs[s][2 * i + 1]) for s in range(args.steps))
-               for i in range(len(problems))]
-    gemm_ms = [statistics.fmean(evs[s][2 * i + 1].elapsed_time(evs[s][2 * i + 2]) for s in range(args.steps))
-               for i in range(len(problems))]
-
+    cast_t = [[] for _ in probs]
+    gemm_t = [[] for _ in probs]
+    for _ in range(min(args.steps, 50)):
+        g_ev.replay()
+        torch.cuda.synchronize(device)
+        for i in range(len(probs)):
+            cast_t[i].append(evs[3 * i].elapsed_time(evs[3 * i + 1]))
+            gemm_t[i].append(evs[3 * i + 1].elapsed_time(evs[3 * i + 2]))
+    cast_ms = [statistics.fmean(v) for v in cast_t]
+    gemm_ms = [statistics.fmean(v) for v in gemm_t]
     ms_max, flops_all = aggregate(local_ms, flops_step, device)
     value = flops_all / (ms_max * 1e-3) / 1e12
 
     # ---------------- e2e through the public API with pinned host buffers ----------------
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    host_bufs = []
-    for (N, K, x, w, c), p in zip(host, problems):
-        ah = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
-        ch = torch.from_numpy(np.ascontiguousarray(c).view(np.int16)).view(torch.bfloat16).pin_memory() \
-            if c is not None else None
-        dh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-        host_bufs.append((ah, ch, dh))
-    h2d = sum(ah.numel() * 2 + (ch.numel() * 2 if ch is not None else 0) for ah, ch, _ in host_bufs)
-    d2h = sum(dh.numel() * 2 for _, _, dh in host_bufs)
+    for p in probs:
+        p["ah"] = torch.from_numpy(np.ascontiguousarray(p["x"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+        p["ch"] = torch.from_numpy(np.ascontiguousarray(p["c"]).view(np.int16)).view(torch.bfloat16).pin_memory() \
+            if p["c"] is not None else None
+        p["dh"] = torch.empty(p["d"].shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(p["ah"].numel() * 2 + (p["ch"].numel() * 2 if p["ch"] is not None else 0) for p in probs)
+    d2h = sum(p["dh"].numel() * 2 for p in probs)
 
     def e2e_step():
-        for (ah, ch, dh), p in zip(host_bufs, problems):
-            p["a"].copy_(ah, non_blocking=True)
-            if ch is not None:
-                p["c"].copy_(ch, non_blocking=True)
+        for p in probs:
+            p["a"].copy_(p["ah"], non_blocking=True)
+            if p["ch"] is not None:
+                p["cd"].copy_(p["ch"], non_blocking=True)
             a_q, sfa = ops.cast_per_token(p["a"], stream=stream)
-            d = ops.fp8_gemm_nt(a_q, sfa, p["b"], p["sfb"], p["c"], out=p["d"], stream=stream)
-            dh.copy_(d, non_blocking=True)
+            if p["kind"] == "dense":
+                d = ops.fp8_gemm_nt(a_q, sfa, p["b"], p["sfb"], p["cd"], out=p["d"], stream=stream)
+            elif p["kind"] == "contiguous":
+                d = ops.m_grouped_fp8_gemm_nt_contiguous(a_q, sfa, p["b"], p["sfb"], p["gl"], p["cd"], out=p["d"],
+                                                         stream=stream)
+            else:
+                d = ops.m_grouped_fp8_gemm_nt_masked(a_q, sfa, p["b"], p["sfb"], p["mm"], p["expected_m"], p["cd"],
+                                                     out=p["d"], stream=stream)
+            p["dh"].copy_(d, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(device)
@@ -335,51 +421,62 @@ def run_cuda(args):
     fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]            # fp8 dense = 2x bf16 (nominal ratio)
     fp8_peak_burst = 2.0 * peaks["bf16_tflops"]
     hbm = peaks["hbm_gbs"]
-    gemm_total_ms = sum(gemm_ms)
-    achieved = sum(2.0 * M * p["N"] * p["K"] for p in problems) / (gemm_total_ms * 1e-3) / 1e12
-    per_shape = []
-    for p, gm, cm in zip(problems, gemm_ms, cast_ms):
-        fl = 2.0 * M * p["N"] * p["K"]
-        by = algorithmic_bytes(M, p["N"], p["K"], with_c)
-        t_tc = fl / (fp8_peak * 1e12)
-        t_hbm = by / (hbm * 1e9)
-        per_shape.append({"N": p["N"], "K": p["K"], "gemm_us": round(gm * 1e3, 2),
-                          "tflops": round(fl / (gm * 1e-3) / 1e12, 1), "gbs": round(by / (gm * 1e-3) / 1e9, 1),
-                          "bound": "tensor" if t_tc >= t_hbm else "hbm",
-                          "roof_frac": round(max(t_tc, t_hbm) / (gm * 1e-3), 3),
-                          "cast_us": round(cm * 1e3, 2),
-                          "cast_gbs": round(cast_bytes(M, p["K"]) / (cm * 1e-3) / 1e9, 1)})
-    traffic = None
+    per_problem = []
+    t_roof_total = 0.0
+    for p, gm, cm in zip(probs, gemm_ms, cast_ms):
+        t_tc = p["flops"] / (fp8_peak * 1e12)
+        t_hbm = p["bytes"] / (hbm * 1e9)
+        t_roof_total += max(t_tc, t_hbm)
+        per_problem.append({"N": p["N"], "K": p["K"], "gemm_us": round(gm * 1e3, 2),
+                            "tflops": round(p["flops"] / (gm * 1e-3) / 1e12, 1),
+                            "gbs": round(p["bytes"] / (gm * 1e-3) / 1e9, 1),
+                            "bound": "tensor" if t_tc >= t_hbm else "hbm",
+                            "roof_frac": round(max(t_tc, t_hbm) / (gm * 1e-3), 3),
+                            "cast_us": round(cm * 1e3, 2),
+                            "cast_gbs": round(cast_bytes(p) / (cm * 1e-3) / 1e9, 1)})
+    gemm_total_s = sum(gemm_ms) * 1e-3
+    flops_sum = sum(p["flops"] for p in probs)
+    bytes_sum = sum(p["bytes"] for p in probs)
+    if flops_sum / (fp8_peak * 1e12) >= bytes_sum / (hbm * 1e9):
+        achieved = flops_sum / gemm_total_s / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / fp8_peak, 4),
+                "peak_source": f"{peaks_src}: 2 x bf16_tflops_sustained (fp8 = 2x bf16 nominal ratio)",
+                "frac_of_burst_peak": round(achieved / fp8_peak_burst, 4)}
+    else:
+        achieved = bytes_sum / gemm_total_s / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": round(hbm, 1), "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "peak_source": f"{peaks_src}: hbm_gbs (copy bandwidth)"}
+    roof["roofline_time_frac"] = round(t_roof_total / gemm_total_s, 4)
+    roof["kernel"] = f"gemm_kernel ({len(probs)} problems, aggregate over launches)"
+    roof["traffic"] = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
         with open(tpath) as f:
-            traffic = json.load(f).get(args.workload)
+            roof["traffic"] = json.load(f).get(args.workload)
 
-    clocks = clk.summary()
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
-        "config": {"workload": wl["desc"], "M": M, "shapes_NK": [list(s) for s in wl["shapes"]],
-                   "step": "per-token cast of A + GEMM D=C+A·Bᵀ per shape; weights cast offline",
+        "config": {"workload": wl["desc"], "shapes_NK": [list(s) for s in wl["shapes"]],
+                   "step": "per-token cast of A + GEMM per problem; weights cast offline",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "no flush: one step's working set is far above the 126 MB L2"},
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp8_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4), "traffic": traffic,
-                     "kernel": "gemm_normal_kernel (6 shapes, aggregate)",
-                     "peak_source": f"{peaks_src}: 2 x bf16_tflops_sustained (fp8 = 2x bf16 nominal ratio)",
-                     "frac_of_burst_peak": round(achieved / fp8_peak_burst, 4)},
-        "per_shape": per_shape,
+                   "l2": ("256 MB flush at the start of every step" if flush is not None
+                          else "no flush: one step's working set is far above the 126 MB L2")},
+        "roofline": roof,
+        "per_problem": per_problem,
         "weight_cast": {"gbs": round(sum(b for _, b in wc_ms) / (sum(t for t, _ in wc_ms) * 1e-3) / 1e9, 1),
                         "ms_total": round(sum(t for t, _ in wc_ms), 3)},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
-                "path": "pinned host A,C -> device, ops.cast_per_token + ops.fp8_gemm_nt, D -> pinned host"},
+                "path": "pinned host activations (and C) -> device, ops cast + GEMM, D -> pinned host"},
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks,
+        "launch": "each step replays a CUDA graph of its launches",
+        "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(wl, host, target_s=args.cpu_seconds)
+        result["cpu_baseline"] = cpu_baseline(wl, probs, target_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -391,37 +488,46 @@ def run_cuda(args):
 # oracle (CPU) arm and baseline
 # ------------------------------------------------------------------------------------------------
 
-def oracle_sample(wl, host, rows: int, cols: int):
-    """Times the oracle on `rows` rows x `cols` columns of every shape (cast of those rows of A
-    plus the GEMM); the weight cast is untimed setup, as in the CUDA arm. Returns (s, flops)."""
+def oracle_sample(probs, rows: int, cols: int):
+    """Times the oracle on `rows` rows x `cols` columns of every problem: the per-token cast of
+    those activation rows and their fp64 GEMM against the matching weights (expert 0 for the
+    grouped layouts, whose first rows belong to it). The weight cast is untimed setup, as in
+    the CUDA arm. Returns (seconds, flops)."""
     import numpy as np
 
     import oracle
     total_s, total_flops = 0.0, 0.0
-    for (N, K, x, w, c) in host:
-        ncol = max(128, min(N, cols // 128 * 128)) if N >= 128 else N
+    for p in probs:
+        N, K = p["N"], p["K"]
+        ncol = N if N < 128 else max(128, min(N, cols // 128 * 128))
+        w = p["w"] if p["kind"] == "dense" else p["w"][0]
+        if p["kind"] == "masked":
+            x, avail = p["x"][0], int(p["masked_m"][0])
+        elif p["kind"] == "contiguous":
+            x, avail = p["x"], int((p["layout"] == 0).sum())
+        else:
+            x, avail = p["x"], p["x"].shape[0]
+        r = max(1, min(rows, avail))
         b, sfb = oracle.cast_per_block(w[:ncol])
-        xr = np.ascontiguousarray(x[:rows])
-        cr = np.ascontiguousarray(c[:rows, :ncol]) if c is not None else None
+        xr = np.ascontiguousarray(x[:r])
+        cr = np.ascontiguousarray(p["c"][:r, :ncol]) if p["c"] is not None else None
         t0 = time.perf_counter()
         a, sfa = oracle.cast_per_token(xr)
         oracle.gemm_nt(a, sfa, b, sfb, cr)
         total_s += time.perf_counter() - t0
-        total_flops += 2.0 * rows * ncol * K
+        total_flops += 2.0 * r * ncol * K
     return total_s, total_flops
 
 
-def cpu_baseline(wl, host, target_s=15.0):
+def cpu_baseline(wl, probs, target_s=15.0):
     import oracle
-    s, f = oracle_sample(wl, host, 1, 1024)                    # calibration probe
+    s, f = oracle_sample(probs, 1, 1024)                      # calibration probe
     rate = f / max(s, 1e-6)
-    # rows x full N per shape, sized to about target_s of CPU work
-    full_cols = max(N for N, _ in wl["shapes"])
-    per_row = sum(2.0 * min(N, full_cols) * K for N, K in wl["shapes"])
-    rows = int(max(1, min(wl["M"], target_s * rate / per_row)))
-    s, f = oracle_sample(wl, host, rows, full_cols)
+    per_row = sum(2.0 * p["N"] * p["K"] for p in probs)
+    rows = int(max(1, min(64 if wl["kind"] == "masked" else 4096, target_s * rate / per_row)))
+    s, f = oracle_sample(probs, rows, max(p["N"] for p in probs))
     return {"value": round(f / s / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"first {rows} rows of A x all N columns of each of the {len(wl['shapes'])} shapes "
+            "sample": f"first {rows} activation rows x all N columns of each of the {len(probs)} problems "
                       f"(per-token cast of those rows + fp64 GEMM), {s:.1f} s on the host"}
 
 
@@ -432,28 +538,28 @@ def run_reference(args):
     import oracle
     oracle.build()
     wl = WORKLOADS[args.workload]
-    host = make_inputs(wl)
-    s, f = oracle_sample(wl, host, 1, 256)
+    probs = make_problems(wl)
+    s, f = oracle_sample(probs, 1, 256)
     rate = f / max(s, 1e-6)
     budget = max(0.02, 120.0 / max(1, args.steps + args.warmup))   # whole run within ~2 minutes
-    per_row_col = sum(2.0 * K for _, K in wl["shapes"])
+    per_row_col = sum(2.0 * p["K"] for p in probs)
     cells = max(128.0, budget * rate / per_row_col)
-    cols = int(min(max(N for N, _ in wl["shapes"]), max(128, cells // 128 * 128)))
-    rows = int(max(1, min(wl["M"], cells / cols)))
+    cols = int(min(max(p["N"] for p in probs), max(128, cells // 128 * 128)))
+    rows = int(max(1, cells / cols))
     for _ in range(args.warmup):
-        oracle_sample(wl, host, rows, cols)
+        oracle_sample(probs, rows, cols)
     tot_s = tot_f = 0.0
     for _ in range(args.steps):
-        s, f = oracle_sample(wl, host, rows, cols)
+        s, f = oracle_sample(probs, rows, cols)
         tot_s += s
         tot_f += f
     value = tot_f / tot_s / 1e12
-    sample = (f"{rows} rows x {cols} columns (capped at N) of each of the {len(wl['shapes'])} shapes per step: "
+    sample = (f"up to {rows} rows x {cols} columns (capped at N) of each of the {len(probs)} problems per step: "
               f"per-token cast of those rows + fp64 GEMM on the host")
     out = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(tot_s / args.steps * 1e3, 3), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-           "config": {"workload": wl["desc"], "M": wl["M"], "shapes_NK": [list(s) for s in wl["shapes"]]},
+           "config": {"workload": wl["desc"], "shapes_NK": [list(s) for s in wl["shapes"]]},
            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
                             "kind": "oracle", "sample": sample},
            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

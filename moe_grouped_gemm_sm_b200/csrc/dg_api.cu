@@ -13,6 +13,7 @@
 #include "../../include/dg.h"
 #include "dg_cast.cuh"
 #include "dg_gemm.cuh"
+#include "dg_gemm_swap.cuh"
 
 namespace {
 
@@ -99,6 +100,18 @@ int forced_pair() {
     if (v == -2) {
         v = -1;
         if (const char *s = std::getenv("DG_FORCE_PAIR")) v = std::atoi(s) ? 1 : 0;
+        cached.store(v);
+    }
+    return v;
+}
+
+// Few-row kernel override for experiments (DG_FORCE_SWAP=0|1); -1 = heuristic.
+int forced_swap() {
+    static std::atomic<int> cached{-2};
+    int v = cached.load();
+    if (v == -2) {
+        v = -1;
+        if (const char *s = std::getenv("DG_FORCE_SWAP")) v = std::atoi(s) ? 1 : 0;
         cached.store(v);
     }
     return v;
@@ -276,6 +289,162 @@ dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *
     return launch_gemm<128, 5, KIND, false>(mp, p, tiles, di, st);
 }
 
+// ---- few-row GEMMs: swapped operands, split-K over a cluster (dg_gemm_swap.cuh) ----
+struct SwapMaps {
+    CUtensorMap w, x, sfa, c;
+};
+
+bool build_swap_maps(SwapMaps &mp, const void *a, const float *sfa, const void *b, const void *c, int rows, int N,
+                     int K, int G, int tn, bool batched) {
+    const uint64_t Gg = static_cast<uint64_t>(G);
+    {   // weights: e4m3 [G][N][K], box 128 x 128 x 1
+        const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), Gg};
+        const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(K) * N};
+        const uint32_t box[3] = {128, 128, 1};
+        if (!encode(&mp.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return false;
+    }
+    {   // activations: e4m3 [G?][rows][K], box 128 x tn
+        const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows), Gg};
+        const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(K) * rows};
+        const uint32_t box[3] = {128, static_cast<uint32_t>(tn), 1};
+        if (!encode(&mp.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, batched ? 3 : 2, a, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return false;
+    }
+    {   // sfa: fp32 [G?][Kb][pad4(rows)], box tn x 1
+        const uint64_t Kb = static_cast<uint64_t>(K / 128), ld = static_cast<uint64_t>(pad4(rows));
+        const uint64_t dims[3] = {ld, Kb, Gg};
+        const uint64_t str[2] = {ld * 4, ld * 4 * Kb};
+        const uint32_t box[3] = {static_cast<uint32_t>(tn), 1, 1};
+        if (!encode(&mp.sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, batched ? 3 : 2, sfa, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+            return false;
+    }
+    if (c) {   // C: bf16 [G?][rows][N], box 128 columns x tn rows (no swizzle: 256-byte rows)
+        const uint64_t dims[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(rows), Gg};
+        const uint64_t str[2] = {static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(N) * 2 * rows};
+        const uint32_t box[3] = {128, static_cast<uint32_t>(tn), 1};
+        if (!encode(&mp.c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, batched ? 3 : 2, c, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+            return false;
+    } else {
+        mp.c = mp.sfa;   // never read when has_c == 0
+    }
+    return true;
+}
+
+// Split count. S = 1: persistent CTAs stride over the tiles, cost ~ ceil(tiles/SMs) · Kb + 2.
+// S > 1 (a power of two <= 8, each split keeping >= 2 K blocks): one cluster per tile, cost ~
+// waves · (Kb/S + 4), the 4 standing for a cluster's fill and its reduction; a wave is as many
+// S-CTA clusters as can be resident at once (capacity[log2 S]).
+int choose_splits(int active_tiles, int Kb, const int *capacity) {
+    int best = 1;
+    double best_cost = static_cast<double>((active_tiles + capacity[0] - 1) / capacity[0]) * Kb + 2;
+    for (int S = 2, i = 1; S <= 8; S *= 2, ++i) {
+        if ((Kb + S - 1) / S < 2) break;
+        if (capacity[i] <= 0) continue;
+        const int waves = (active_tiles + capacity[i] - 1) / capacity[i];
+        const double cost = static_cast<double>(waves) * ((Kb + S - 1) / S + 4);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = S;
+        }
+    }
+    return best;
+}
+
+struct SwapKernelInfo {
+    std::atomic<int> ready{0};
+    int capacity[4] = {0, 0, 0, 0};   // resident clusters of 1, 2, 4, 8 CTAs
+};
+
+template <int TN, int STAGES, int KIND>
+dg_status launch_swap(const SwapMaps &mp, dg::SwapParams &p, int tiles, int active, const DeviceInfo *di,
+                      cudaStream_t st) {
+    using L = dg::SwapLayout<TN, STAGES>;
+    auto kern = dg::gemm_swap_kernel<TN, STAGES, KIND>;
+    static SwapKernelInfo info[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
+    SwapKernelInfo &ki = info[dev];
+    if (!ki.ready.load()) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!ki.ready.load()) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) != cudaSuccess)
+                return DG_ERR_CUDA;
+            ki.capacity[0] = di->sm_count;
+            for (int i = 1, S = 2; i < 4; ++i, S *= 2) {
+                cudaLaunchConfig_t qc = {};
+                cudaLaunchAttribute qa[1];
+                qc.gridDim = dim3(S * 16, 1, 1);
+                qc.blockDim = dim3(L::THREADS, 1, 1);
+                qc.dynamicSmemBytes = L::ALLOC;
+                qa[0].id = cudaLaunchAttributeClusterDimension;
+                qa[0].val.clusterDim.x = S;
+                qa[0].val.clusterDim.y = 1;
+                qa[0].val.clusterDim.z = 1;
+                qc.attrs = qa;
+                qc.numAttrs = 1;
+                int n = 0;
+                if (cudaOccupancyMaxActiveClusters(&n, kern, &qc) != cudaSuccess) n = 0;
+                ki.capacity[i] = n;
+            }
+            ki.ready.store(1);
+        }
+    }
+    p.splits = choose_splits(active, p.Kb, ki.capacity);
+    p.num_tiles = tiles;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    const int persistent = tiles < di->sm_count ? tiles : di->sm_count;
+    cfg.gridDim = dim3(p.splits > 1 ? tiles * p.splits : persistent, 1, 1);
+    cfg.blockDim = dim3(L::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = L::ALLOC;
+    cfg.stream = st;
+    if (p.splits > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = p.splits;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return from_cuda(cudaLaunchKernelEx(&cfg, kern, mp.w, mp.x, mp.sfa, mp.c, p));
+}
+
+template <int KIND>
+dg_status run_swap(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
+                   const int32_t *masked_m, int expected_m, int rows, int N, int K, int G, cudaStream_t st) {
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    const bool batched = KIND == dg::KIND_MASKED;
+    const int hint = batched ? (expected_m > 0 ? expected_m : rows) : rows;
+    const int tn = hint <= 64 ? 64 : 128;
+    dg::SwapParams p{};
+    p.M = rows;
+    p.N = N;
+    p.K = K;
+    p.G = G;
+    p.Kb = K / 128;
+    p.Nb = (N + 127) / 128;
+    p.ld_sfa = pad4(rows);
+    p.n_tiles = (N + 127) / 128;
+    p.m_tiles = (rows + tn - 1) / tn;
+    p.has_c = c != nullptr;
+    p.sfb = sfb;
+    p.masked_m = masked_m;
+    p.c = static_cast<const __nv_bfloat16 *>(c);
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.err = di->err;
+    p.timeout_ns = wait_limit_ns();
+    const int tiles = (batched ? G : 1) * p.m_tiles * p.n_tiles;
+    const int active = (batched ? G : 1) * ((hint < rows ? hint : rows) + tn - 1) / tn * p.n_tiles;
+    SwapMaps mp;
+    if (!build_swap_maps(mp, a, sfa, b, c, rows, N, K, G, tn, batched)) return DG_ERR_INVALID_ARG;
+    if (tn == 64) return launch_swap<64, 8, KIND>(mp, p, tiles, active, di, st);
+    return launch_swap<128, 5, KIND>(mp, p, tiles, active, di, st);
+}
+
 dg_status check_gemm_common(const void *a, const float *sfa, const void *b, const float *sfb, const void *c,
                             const void *d, int N, int K) {
     if (!a || !sfa || !b || !sfb || !d) return DG_ERR_INVALID_ARG;
@@ -296,6 +465,9 @@ dg_status dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const f
     dg_status s = check_gemm_common(a, sfa, b, sfb, c, d, N, K);
     if (s != DG_OK) return s;
     if (M == 0) return DG_OK;
+    const int fs = forced_swap();
+    if (fs >= 0 ? fs == 1 && M <= 128 : M <= 128)
+        return run_swap<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, 0, M, N, K, 1, static_cast<cudaStream_t>(stream));
     return run_gemm<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, nullptr, M, N, K, 1,
                                     static_cast<cudaStream_t>(stream));
 }
@@ -314,11 +486,13 @@ dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, c
 dg_status dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb,
                                           const void *c, void *d, const int32_t *masked_m, int expected_m, int G,
                                           int M_max, int N, int K, void *stream) {
-    (void)expected_m;
     if (G <= 0 || M_max < 0 || !masked_m || expected_m < 0) return DG_ERR_INVALID_ARG;
     dg_status s = check_gemm_common(a, sfa, b, sfb, c, d, N, K);
     if (s != DG_OK) return s;
     if (M_max == 0) return DG_OK;
+    if (forced_swap() != 0)
+        return run_swap<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, masked_m, expected_m, M_max, N, K, G,
+                                         static_cast<cudaStream_t>(stream));
     return run_gemm<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, nullptr, masked_m, M_max, N, K, G,
                                      static_cast<cudaStream_t>(stream));
 }
