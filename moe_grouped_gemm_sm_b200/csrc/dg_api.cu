@@ -490,7 +490,7 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const
     dg_status s = check_gemm_common(a, sfa, b, sfb, c, d, N, K);
     if (s != DG_OK) return s;
     if (M_max == 0) return DG_OK;
-    if (forced_swap() != 0)
+    if (forced_swap() == 1)   // the pair kernel streams the masked page shapes faster
         return run_swap<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, masked_m, expected_m, M_max, N, K, G,
                                          static_cast<cudaStream_t>(stream));
     return run_gemm<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, nullptr, masked_m, M_max, N, K, G,

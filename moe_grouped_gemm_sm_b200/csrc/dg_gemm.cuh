@@ -25,8 +25,9 @@
 //               warpgroup j owns columns [j·BN/2, (j+1)·BN/2). Per K block: wait for the TMEM
 //               buffer, load the partial in 32-column batches (the next batch in flight while
 //               the previous one is folded in), release the buffer, acc = fma(p, sa·sb, acc).
-//               sfa comes straight from global memory three K blocks ahead, sfb one 32-K-block
-//               window per lane. Epilogue: C (prefetched by TMA at tile start) is added, the
+//               sfa arrives by TMA in a ring of its own (one BM-float column per K block,
+//               loaded by the producer ahead of the operands), sfb one 32-K-block window per
+//               lane broadcast by shuffle. Epilogue: C (prefetched by TMA at tile start) is added, the
 //               result converted to bf16 (round to nearest even) into a 128-byte-swizzled slab
 //               and stored by TMA.
 //
