@@ -13,14 +13,14 @@
 //                 rows of the partial. Per SM this halves the B bytes that cross L2 -> SMEM.
 //
 // CTA layout (384 threads, one CTA per SM, persistent over tiles):
-//   warp 0      TMA producer: A tile [128 x 128 B] and B tile [BN or BN/2 x 128 B] into a
-//               STAGES-deep ring guarded by full/empty mbarriers (for a pair, both CTAs' loads
-//               count on the leader's full barrier).
+//   warp 0      TMA producer of A: A tile [128 x 128 B] into a STAGES-deep ring guarded by
+//               full/empty mbarriers (for a pair, both CTAs' loads count on the leader's full
+//               barrier); it also arms each stage's expected bytes.
 //   warp 1      TMEM allocator and (leader only) the single thread that issues tcgen05.mma
 //               kind::f8f6f4, four K=32 steps per K block, into one of 512/BN TMEM buffers, and
 //               commits the stage (empty) and the buffer (tfull) — to both CTAs of a pair.
-//   warp 2      (contiguous pair tiles) lists the pairs once in the prologue; otherwise idle.
-//   warp 3      idle.
+//   warp 2      loads B (and, for contiguous pair tiles, first lists the pairs once).
+//   warp 3      loads the A-scale ring.
 //   warps 4-11  two math warpgroups. Warp w reads TMEM lanes 32·(w%4)..+31 (its 32 rows);
 //               warpgroup j owns columns [j·BN/2, (j+1)·BN/2). Per K block: wait for the TMEM
 //               buffer, load the partial in 32-column batches (the next batch in flight while
@@ -327,13 +327,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
     if (warp < 4) {
         reg_dealloc<56>();
-        if (warp == 0 && lane == 0) {
-            // ---------------- TMA producer ----------------
+        // TMA producers, one thread per stream: warp 0 arms each stage and loads A, warp 2 loads
+        // B, warp 3 loads the A scales. One thread's bulk copies are served one after another
+        // (a fixed cost per copy, whatever its size), so three streams keep three in flight.
+        // All three wait on the same "empty" barrier of the ring; none can run more than
+        // STAGES K blocks ahead of the others, since a stage is only freed once all its loads
+        // have landed and the MMA has consumed it.
+        const int stream = warp == 0 ? 0 : (warp == 2 ? 1 : (warp == 3 ? 2 : -1));
+        if (stream >= 0 && lane == 0) {
             uint32_t it = 0;
             for (int t = cid; t < num_tiles && !*abort_flag; t += ncid) {
                 const TileInfo ti = decode_tile<KIND, PAIR>(t, p, pair_first, num_pairs, rank);
                 if (!ti.valid) {
-                    if (KIND == KIND_CONTIGUOUS && ti.g >= p.G) report_error(p.err, ERR_DATA);
+                    if (stream == 0 && KIND == KIND_CONTIGUOUS && ti.g >= p.G) report_error(p.err, ERR_DATA);
                     continue;
                 }
                 const int brow = ti.n_blk * BN + static_cast<int>(rank) * L::B_ROWS;
@@ -341,30 +347,39 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!mbar_wait(&empty[s], ph ^ 1, ctx)) break;
-                    const int j = it % L::SFS;
-                    float *sf = reinterpret_cast<float *>(smem + L::OFF_SFA) + j * BM;
-                    mbar_arrive_expect_tx(&sfa_full[j], BM * 4);
-                    if (KIND == KIND_MASKED)
-                        tma_load_3d(&tm_sfa, &sfa_full[j], sf, ti.row0, kb, ti.g);
-                    else
-                        tma_load_2d(&tm_sfa, &sfa_full[j], sf, ti.row0, kb);
+                    if (stream == 2) {
+                        const int j = it % L::SFS;
+                        float *sf = reinterpret_cast<float *>(smem + L::OFF_SFA) + j * BM;
+                        mbar_arrive_expect_tx(&sfa_full[j], BM * 4);
+                        if (KIND == KIND_MASKED)
+                            tma_load_3d(&tm_sfa, &sfa_full[j], sf, ti.row0, kb, ti.g);
+                        else
+                            tma_load_2d(&tm_sfa, &sfa_full[j], sf, ti.row0, kb);
+                        continue;
+                    }
                     uint8_t *sa = smem + L::OFF_A + s * L::A_BYTES;
                     uint8_t *sb = smem + L::OFF_B + s * L::B_BYTES;
                     if (PAIR) {
                         const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);   // the leader's barrier
-                        if (leader) mbar_arrive_expect_tx(&full[s], L::STAGE_TX);
-                        if (KIND == KIND_MASKED)
-                            tma_load_3d_pair(&tm_a, fb, sa, kb * BK, ti.row0, ti.g);
-                        else
-                            tma_load_2d_pair(&tm_a, fb, sa, kb * BK, ti.row0);
-                        tma_load_3d_pair(&tm_b, fb, sb, kb * BK, brow, ti.g);
+                        if (stream == 0) {
+                            if (leader) mbar_arrive_expect_tx(&full[s], L::STAGE_TX);
+                            if (KIND == KIND_MASKED)
+                                tma_load_3d_pair(&tm_a, fb, sa, kb * BK, ti.row0, ti.g);
+                            else
+                                tma_load_2d_pair(&tm_a, fb, sa, kb * BK, ti.row0);
+                        } else {
+                            tma_load_3d_pair(&tm_b, fb, sb, kb * BK, brow, ti.g);
+                        }
                     } else {
-                        mbar_arrive_expect_tx(&full[s], L::STAGE_TX);
-                        if (KIND == KIND_MASKED)
-                            tma_load_3d(&tm_a, &full[s], sa, kb * BK, ti.row0, ti.g);
-                        else
-                            tma_load_2d(&tm_a, &full[s], sa, kb * BK, ti.row0);
-                        tma_load_3d(&tm_b, &full[s], sb, kb * BK, brow, ti.g);
+                        if (stream == 0) {
+                            mbar_arrive_expect_tx(&full[s], L::STAGE_TX);
+                            if (KIND == KIND_MASKED)
+                                tma_load_3d(&tm_a, &full[s], sa, kb * BK, ti.row0, ti.g);
+                            else
+                                tma_load_2d(&tm_a, &full[s], sa, kb * BK, ti.row0);
+                        } else {
+                            tma_load_3d(&tm_b, &full[s], sb, kb * BK, brow, ti.g);
+                        }
                     }
                 }
             }

@@ -16,9 +16,9 @@
 //     No global workspace is used and the reduction order is fixed (deterministic);
 //   * a deep TMA ring (6-8 stages of the 16 KB weight tile) keeps enough bytes in flight.
 //
-// CTA layout: warp 0 TMA producer, warp 1 TMEM allocator + single-thread tcgen05.mma issuer
-// (kind::f8f6f4, M = 128, N = TN), warps 2-3 idle, warps 4.. TN/64 math warpgroups (thread =
-// weight row, registers = its warpgroup's 64 token columns).
+// CTA layout: warps 0, 2, 3 TMA producers (weights, activations, A scales), warp 1 TMEM
+// allocator + single-thread tcgen05.mma issuer (kind::f8f6f4, M = 128, N = TN), warps 4.. TN/64
+// math warpgroups (thread = weight row, registers = its warpgroup's 64 token columns).
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -167,8 +167,11 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
     int g = 0, m0 = 0, n0 = 0, rows = 0;                   // the last tile (split reduction)
 
     if (warp < 4) {
-        if (warp == 0 && lane == 0) {
-            // ---------------- TMA producer ----------------
+        // TMA producers, one thread per stream (one thread's bulk copies are served one after
+        // another): warp 0 arms each stage and loads the weights, warp 2 the activations,
+        // warp 3 the A scales. All wait on the ring's "empty" barriers.
+        const int stream = warp == 0 ? 0 : (warp == 2 ? 1 : (warp == 3 ? 2 : -1));
+        if (stream >= 0 && lane == 0) {
             uint32_t it = 0;
             for (int t = cid; t < p.num_tiles && !*abort_flag; t += ncid) {
                 int tg, tm0, tn0;
@@ -177,19 +180,22 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
                     const int kb = kb0 + i;
                     const int s = it % STAGES;
                     if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, ctx)) break;
-                    const int j = it % L::SFS;
-                    mbar_arrive_expect_tx(&sfa_full[j], TN * 4);
-                    float *sf = reinterpret_cast<float *>(smem + L::OFF_SFA) + j * TN;
-                    if (KIND == KIND_MASKED)
-                        tma_load_3d(&tm_sfa, &sfa_full[j], sf, tm0, kb, tg);
-                    else
-                        tma_load_2d(&tm_sfa, &sfa_full[j], sf, tm0, kb);
-                    mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
-                    tma_load_3d(&tm_w, &full[s], smem + L::OFF_W + s * L::W_BYTES, kb * BK, tn0, tg);
-                    if (KIND == KIND_MASKED)
+                    if (stream == 2) {
+                        const int j = it % L::SFS;
+                        mbar_arrive_expect_tx(&sfa_full[j], TN * 4);
+                        float *sf = reinterpret_cast<float *>(smem + L::OFF_SFA) + j * TN;
+                        if (KIND == KIND_MASKED)
+                            tma_load_3d(&tm_sfa, &sfa_full[j], sf, tm0, kb, tg);
+                        else
+                            tma_load_2d(&tm_sfa, &sfa_full[j], sf, tm0, kb);
+                    } else if (stream == 0) {
+                        mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
+                        tma_load_3d(&tm_w, &full[s], smem + L::OFF_W + s * L::W_BYTES, kb * BK, tn0, tg);
+                    } else if (KIND == KIND_MASKED) {
                         tma_load_3d(&tm_x, &full[s], smem + L::OFF_X + s * L::X_BYTES, kb * BK, tm0, tg);
-                    else
+                    } else {
                         tma_load_2d(&tm_x, &full[s], smem + L::OFF_X + s * L::X_BYTES, kb * BK, tm0);
+                    }
                 }
             }
         } else if (warp == 1 && lane == 0) {

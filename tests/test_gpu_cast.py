@@ -74,3 +74,56 @@ def test_cast_then_transform_roundtrip(oracle):
     _, sfa = ops.cast_per_token(bf16_dev(x))
     kmajor = sfa[:, :50].t().contiguous()
     assert torch.equal(ops.transform_sf(kmajor)[:, :50], sfa[:, :50])
+
+
+def _all_finite_bf16(limit: float) -> np.ndarray:
+    """Every finite bf16 bit pattern (both signs, both zeros) whose magnitude is <= limit."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    finite = (bits & 0x7F80) != 0x7F80
+    mag = synth.bf16_bits_to_f32(bits & 0x7FFF)
+    return bits[finite & (mag <= np.float32(limit))]
+
+
+# amax values: ordinary ones, one whose scale is a subnormal fp32 (1/s still finite), one
+# whose scale is so small that 1/s overflows, a huge one, and a bf16 subnormal amax.
+SWEEP_AMAX = [1.0, 3.1875, 0.3, 57.75, 1.0e30, 448.0 * 2.0 ** -127, 2.0 ** -126, 2.0 ** -133]
+
+
+@pytest.mark.parametrize("amax", SWEEP_AMAX)
+def test_cast_per_token_every_bf16_value(oracle, amax):
+    """Each row's K slice holds the amax first, then a run of the sweep of every finite bf16
+    value up to that magnitude: every code decision of the cast for that scale is checked."""
+    a_bits = np.uint16(synth.f32_to_bf16_bits(np.array([amax], np.float32))[0])
+    amax_f = float(synth.bf16_bits_to_f32(np.array([a_bits], np.uint16))[0])
+    vals = _all_finite_bf16(amax_f)
+    rows = (vals.size + 126) // 127
+    x = np.zeros((rows, 128), np.uint16)
+    flat = np.zeros(rows * 127, np.uint16)
+    flat[:vals.size] = vals
+    x[:, 0] = a_bits
+    x[:, 1:] = flat.reshape(rows, 127)
+    q, sfa = ops.cast_per_token(bf16_dev(x))
+    torch.cuda.synchronize()
+    qo, so = oracle.cast_per_token(x)
+    assert np.array_equal(host(q), qo)
+    assert np.array_equal(host(sfa)[:, :rows].view(np.uint32), so[:, :rows].view(np.uint32))
+
+
+@pytest.mark.parametrize("amax", [3.1875, 448.0 * 2.0 ** -127, 1.0e30])
+def test_cast_per_block_every_bf16_value(oracle, amax):
+    a_bits = np.uint16(synth.f32_to_bf16_bits(np.array([amax], np.float32))[0])
+    amax_f = float(synth.bf16_bits_to_f32(np.array([a_bits], np.uint16))[0])
+    vals = _all_finite_bf16(amax_f)
+    per_block = 128 * 128 - 1
+    nblk = (vals.size + per_block - 1) // per_block
+    w = np.zeros((nblk * 128, 128), np.uint16)
+    flat = np.zeros(nblk * per_block, np.uint16)
+    flat[:vals.size] = vals
+    for b in range(nblk):
+        blk = np.concatenate([np.array([a_bits], np.uint16), flat[b * per_block:(b + 1) * per_block]])
+        w[b * 128:(b + 1) * 128] = blk.reshape(128, 128)
+    q, sfb = ops.cast_per_block(bf16_dev(w))
+    torch.cuda.synchronize()
+    qo, so = oracle.cast_per_block(w)
+    assert np.array_equal(host(q), qo)
+    assert np.array_equal(host(sfb).view(np.uint32), so.view(np.uint32))
