@@ -519,10 +519,19 @@ dg_status dg_cast_fp8_per_token(const void *x, void *q, float *sfa, int batch, i
     dg_status s = device_info(&di);
     if (s != DG_OK) return s;
     const int Kb = K / 128;
-    dim3 grid((M + 31) / 32, (Kb + 3) / 4, batch);
-    if (grid.y > 65535) return DG_ERR_INVALID_ARG;
-    dg::cast_per_token_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const __nv_bfloat16 *>(x), static_cast<uint8_t *>(q), sfa, M, K, pad4(M));
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long long big_blocks = static_cast<long long>((M + 31) / 32) * ((Kb + 3) / 4) * batch;
+    if (big_blocks >= 2LL * di->sm_count) {   // enough 32 x 4 blocks for two per SM
+        dim3 grid((M + 31) / 32, (Kb + 3) / 4, batch);
+        if (grid.y > 65535) return DG_ERR_INVALID_ARG;
+        dg::cast_per_token_kernel<32, 4><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x),
+                                                                 static_cast<uint8_t *>(q), sfa, M, K, pad4(M));
+    } else {
+        dim3 grid((M + 7) / 8, (Kb + 1) / 2, batch);
+        if (grid.y > 65535) return DG_ERR_INVALID_ARG;
+        dg::cast_per_token_kernel<8, 2><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x),
+                                                                static_cast<uint8_t *>(q), sfa, M, K, pad4(M));
+    }
     return from_cuda(cudaGetLastError());
 }
 

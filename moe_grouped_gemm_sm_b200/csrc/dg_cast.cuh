@@ -59,36 +59,42 @@ __device__ __forceinline__ uint2 quant8(const float (&f)[8], float s) {
     return make_uint2(w[0], w[1]);
 }
 
-// Per-token cast. Block: 256 threads = 8 warps covering 32 rows x 4 K-slices of one batch
-// entry. Each warp owns 4 rows; one warp-wide load covers two slices of one row (lanes 0-15
-// slice 2i, lanes 16-31 slice 2i+1, 16 bytes per lane), and all 8 loads of a thread are issued
-// before any is used. Grid: (ceil(M/32), ceil(Kb/4), batch).
+// Per-token cast. Block: 256 threads covering ROWS rows x KBS K-slices of one batch entry, in
+// "slice halves": a half-warp covers one row's 128-value slice (16 lanes x 8 values, 16 bytes
+// per lane). Slice s = i·16 + warp·2 + half (i < ROWS·KBS/16) is row s / KBS, slice s % KBS, so
+// that one warp-wide load covers two adjacent slices of one row (512 contiguous bytes). All
+// loads of a thread are issued before any is used. Two shapes: 32 x 4 (8 slices per thread,
+// many bytes in flight per thread) for many rows, 8 x 2 (one slice per thread, 16x the blocks)
+// for few rows, where each block's serial chain of divisions would otherwise set the time.
+// Grid: (ceil(M/ROWS), ceil(Kb/KBS), batch).
+template <int ROWS, int KBS>
 __global__ void __launch_bounds__(256) cast_per_token_kernel(const __nv_bfloat16 *__restrict__ x,
                                                              uint8_t *__restrict__ q, float *__restrict__ sfa,
                                                              int M, int K, int ld) {
-    __shared__ float s_sf[4][32];
+    constexpr int PER = ROWS * KBS / 16;
+    static_assert(PER >= 1 && ROWS * KBS % 16 == 0 && KBS % 2 == 0, "block shape");
+    __shared__ float s_sf[KBS][ROWS];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int half = lane >> 4, hl = lane & 15;
     const int Kb = K >> 7;
     const size_t bofs = static_cast<size_t>(blockIdx.z) * M;
-    const int r0 = blockIdx.x * 32, kb0 = blockIdx.y * 4;
+    const int r0 = blockIdx.x * ROWS, kb0 = blockIdx.y * KBS;
 
-    uint4 v[8];
+    uint4 v[PER];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int row = r0 + warp * 4 + (i >> 1);
-        const int kb = kb0 + (i & 1) * 2 + half;
+    for (int i = 0; i < PER; ++i) {
+        const int sl = i * 16 + warp * 2 + half;
+        const int row = r0 + sl / KBS, kb = kb0 + sl % KBS;
         if (row < M && kb < Kb)
             v[i] = ldg_stream_v4(x + (bofs + row) * K + kb * 128 + hl * 8);
         else
             v[i] = make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int rl = warp * 4 + (i >> 1);
-        const int row = r0 + rl;
-        const int kbl = (i & 1) * 2 + half;
-        const int kb = kb0 + kbl;
+    for (int i = 0; i < PER; ++i) {
+        const int sl = i * 16 + warp * 2 + half;
+        const int rl = sl / KBS, kbl = sl % KBS;
+        const int row = r0 + rl, kb = kb0 + kbl;
         float f[8];
         bf16x8_to_f32(v[i], f);
         float m = amax8(f);
@@ -101,8 +107,8 @@ __global__ void __launch_bounds__(256) cast_per_token_kernel(const __nv_bfloat16
         }
     }
     __syncthreads();
-    if (threadIdx.x < 128) {
-        const int kbl = threadIdx.x >> 5, rr = threadIdx.x & 31;
+    for (int idx = threadIdx.x; idx < ROWS * KBS; idx += 256) {
+        const int kbl = idx / ROWS, rr = idx % ROWS;
         const int row = r0 + rr, kb = kb0 + kbl;
         if (row < M && kb < Kb) sfa[(static_cast<size_t>(blockIdx.z) * Kb + kb) * ld + row] = s_sf[kbl][rr];
     }
