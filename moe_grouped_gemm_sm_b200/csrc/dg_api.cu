@@ -9,6 +9,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/dg.h"
 #include "dg_cast.cuh"
@@ -332,91 +333,87 @@ bool build_swap_maps(SwapMaps &mp, const void *a, const float *sfa, const void *
     return true;
 }
 
-// Split count. S = 1: persistent CTAs stride over the tiles, cost ~ ceil(tiles/SMs) · Kb + 2.
-// S > 1 (a power of two <= 8, each split keeping >= 2 K blocks): one cluster per tile, cost ~
-// waves · (Kb/S + 4), the 4 standing for a cluster's fill and its reduction; a wave is as many
-// S-CTA clusters as can be resident at once (capacity[log2 S]).
-int choose_splits(int active_tiles, int Kb, const int *capacity) {
-    int best = 1;
-    double best_cost = static_cast<double>((active_tiles + capacity[0] - 1) / capacity[0]) * Kb + 2;
-    for (int S = 2, i = 1; S <= 8; S *= 2, ++i) {
-        if ((Kb + S - 1) / S < 2) break;
-        if (capacity[i] <= 0) continue;
-        const int waves = (active_tiles + capacity[i] - 1) / capacity[i];
-        const double cost = static_cast<double>(waves) * ((Kb + S - 1) / S + 4);
-        if (cost < best_cost - 1e-9) {
-            best_cost = cost;
-            best = S;
+// Stream-K workspace of the few-row kernel: fp32 partials [slots][128][128] and one flag per
+// slot, flags zero between launches. One per (device, stream), so that launches on different
+// streams never share flags; allocated on a stream's first few-row call, which must not be
+// under graph capture (the call then takes the tile kernel, which needs no workspace).
+struct SwapWorkspace {
+    int dev = -1;
+    cudaStream_t stream = nullptr;
+    float *ws = nullptr;
+    int *flags = nullptr;
+    int slots = 0;
+};
+std::vector<SwapWorkspace> g_swap_ws;
+
+bool swap_workspace(int dev, int sm_count, cudaStream_t st, SwapWorkspace *out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (const SwapWorkspace &w : g_swap_ws)
+        if (w.dev == dev && w.stream == st) {
+            *out = w;
+            return true;
         }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return false;
+    SwapWorkspace w;
+    w.dev = dev;
+    w.stream = st;
+    w.slots = sm_count;
+    const size_t ws_bytes = static_cast<size_t>(sm_count) * 128 * 128 * sizeof(float);
+    if (cudaMalloc(&w.ws, ws_bytes) != cudaSuccess) return false;
+    if (cudaMalloc(&w.flags, static_cast<size_t>(sm_count) * sizeof(int)) != cudaSuccess ||
+        cudaMemset(w.flags, 0, static_cast<size_t>(sm_count) * sizeof(int)) != cudaSuccess) {
+        cudaFree(w.ws);
+        return false;
     }
-    return best;
+    g_swap_ws.push_back(w);
+    *out = w;
+    return true;
 }
 
-struct SwapKernelInfo {
-    std::atomic<int> ready{0};
-    int capacity[4] = {0, 0, 0, 0};   // resident clusters of 1, 2, 4, 8 CTAs
-};
+// After a device error a launch may have stopped with flags still set: zero this device's.
+void reset_swap_flags(int dev) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (const SwapWorkspace &w : g_swap_ws)
+        if (w.dev == dev) cudaMemset(w.flags, 0, static_cast<size_t>(w.slots) * sizeof(int));
+}
 
 template <int TN, int STAGES, int KIND>
-dg_status launch_swap(const SwapMaps &mp, dg::SwapParams &p, int tiles, int active, const DeviceInfo *di,
+dg_status launch_swap(const SwapMaps &mp, const dg::SwapParams &p, long long tiles, const DeviceInfo *di,
                       cudaStream_t st) {
     using L = dg::SwapLayout<TN, STAGES>;
+    const long long units = tiles * p.Kb;
     auto kern = dg::gemm_swap_kernel<TN, STAGES, KIND>;
-    static SwapKernelInfo info[kMaxDevices];
+    static std::atomic<int> ready[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
-    SwapKernelInfo &ki = info[dev];
-    if (!ki.ready.load()) {
+    if (!ready[dev].load()) {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!ki.ready.load()) {
+        if (!ready[dev].load()) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) != cudaSuccess)
                 return DG_ERR_CUDA;
-            ki.capacity[0] = di->sm_count;
-            for (int i = 1, S = 2; i < 4; ++i, S *= 2) {
-                cudaLaunchConfig_t qc = {};
-                cudaLaunchAttribute qa[1];
-                qc.gridDim = dim3(S * 16, 1, 1);
-                qc.blockDim = dim3(L::THREADS, 1, 1);
-                qc.dynamicSmemBytes = L::ALLOC;
-                qa[0].id = cudaLaunchAttributeClusterDimension;
-                qa[0].val.clusterDim.x = S;
-                qa[0].val.clusterDim.y = 1;
-                qa[0].val.clusterDim.z = 1;
-                qc.attrs = qa;
-                qc.numAttrs = 1;
-                int n = 0;
-                if (cudaOccupancyMaxActiveClusters(&n, kern, &qc) != cudaSuccess) n = 0;
-                ki.capacity[i] = n;
-            }
-            ki.ready.store(1);
+            ready[dev].store(1);
         }
     }
-    p.splits = choose_splits(active, p.Kb, ki.capacity);
-    p.num_tiles = tiles;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    const int persistent = tiles < di->sm_count ? tiles : di->sm_count;
-    cfg.gridDim = dim3(p.splits > 1 ? tiles * p.splits : persistent, 1, 1);
-    cfg.blockDim = dim3(L::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = L::ALLOC;
-    cfg.stream = st;
-    if (p.splits > 1) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = p.splits;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
-    return from_cuda(cudaLaunchKernelEx(&cfg, kern, mp.w, mp.x, mp.sfa, mp.c, p));
+    // one CTA per SM (the shared memory allows one); the kernel cuts the units over as many of
+    // them as its per-tile partial limit allows
+    const long long grid = units < di->sm_count ? units : di->sm_count;
+    if (grid <= 0) return DG_OK;
+    kern<<<static_cast<unsigned>(grid), L::THREADS, L::ALLOC, st>>>(mp.w, mp.x, mp.sfa, mp.c, p);
+    return from_cuda(cudaGetLastError());
 }
 
+// Returns DG_ERR_UNSUPPORTED (nothing launched) when no workspace is available for `st`.
 template <int KIND>
 dg_status run_swap(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
                    const int32_t *masked_m, int expected_m, int rows, int N, int K, int G, cudaStream_t st) {
     const DeviceInfo *di = nullptr;
     dg_status s = device_info(&di);
     if (s != DG_OK) return s;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
+    SwapWorkspace w;
+    if (!swap_workspace(dev, di->sm_count, st, &w)) return DG_ERR_UNSUPPORTED;
     const bool batched = KIND == dg::KIND_MASKED;
     const int hint = batched ? (expected_m > 0 ? expected_m : rows) : rows;
     const int tn = hint <= 64 ? 64 : 128;
@@ -435,14 +432,16 @@ dg_status run_swap(const void *a, const float *sfa, const void *b, const float *
     p.masked_m = masked_m;
     p.c = static_cast<const __nv_bfloat16 *>(c);
     p.d = static_cast<__nv_bfloat16 *>(d);
+    p.ws = w.ws;
+    p.flags = w.flags;
     p.err = di->err;
     p.timeout_ns = wait_limit_ns();
-    const int tiles = (batched ? G : 1) * p.m_tiles * p.n_tiles;
-    const int active = (batched ? G : 1) * ((hint < rows ? hint : rows) + tn - 1) / tn * p.n_tiles;
+    // the largest possible tile set: masked groups may use fewer
+    const long long tiles = static_cast<long long>(batched ? G : 1) * p.m_tiles * p.n_tiles;
     SwapMaps mp;
     if (!build_swap_maps(mp, a, sfa, b, c, rows, N, K, G, tn, batched)) return DG_ERR_INVALID_ARG;
-    if (tn == 64) return launch_swap<64, 8, KIND>(mp, p, tiles, active, di, st);
-    return launch_swap<128, 5, KIND>(mp, p, tiles, active, di, st);
+    if (tn == 64) return launch_swap<64, 8, KIND>(mp, p, tiles, di, st);
+    return launch_swap<128, 5, KIND>(mp, p, tiles, di, st);
 }
 
 dg_status check_gemm_common(const void *a, const float *sfa, const void *b, const float *sfb, const void *c,
@@ -466,8 +465,11 @@ dg_status dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const f
     if (s != DG_OK) return s;
     if (M == 0) return DG_OK;
     const int fs = forced_swap();
-    if (fs >= 0 ? fs == 1 && M <= 128 : M <= 128)
-        return run_swap<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, 0, M, N, K, 1, static_cast<cudaStream_t>(stream));
+    if (fs >= 0 ? fs == 1 && M <= 128 : M <= 128) {
+        const dg_status r = run_swap<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, 0, M, N, K, 1,
+                                                     static_cast<cudaStream_t>(stream));
+        if (r != DG_ERR_UNSUPPORTED) return r;
+    }
     return run_gemm<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, nullptr, M, N, K, 1,
                                     static_cast<cudaStream_t>(stream));
 }
@@ -490,9 +492,11 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const
     dg_status s = check_gemm_common(a, sfa, b, sfb, c, d, N, K);
     if (s != DG_OK) return s;
     if (M_max == 0) return DG_OK;
-    if (forced_swap() == 1)   // the pair kernel streams the masked page shapes faster
-        return run_swap<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, masked_m, expected_m, M_max, N, K, G,
-                                         static_cast<cudaStream_t>(stream));
+    if (forced_swap() == 1) {   // the pair kernel streams the masked page shapes faster
+        const dg_status r = run_swap<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, masked_m, expected_m, M_max, N, K, G,
+                                                      static_cast<cudaStream_t>(stream));
+        if (r != DG_ERR_UNSUPPORTED) return r;
+    }
     return run_gemm<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, nullptr, masked_m, M_max, N, K, G,
                                      static_cast<cudaStream_t>(stream));
 }
@@ -561,6 +565,8 @@ dg_status dg_get_device_error(void *stream) {
     if (v != 0) {
         const int zero = 0;
         if (cudaMemcpy(di->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return DG_ERR_CUDA;
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess) reset_swap_flags(dev);
     }
     if (v == dg::ERR_TIMEOUT) return DG_ERR_TIMEOUT;
     if (v != 0) return DG_ERR_DEVICE;

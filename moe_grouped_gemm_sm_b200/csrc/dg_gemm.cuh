@@ -13,14 +13,15 @@
 //                 rows of the partial. Per SM this halves the B bytes that cross L2 -> SMEM.
 //
 // CTA layout (384 threads, one CTA per SM, persistent over tiles):
-//   warp 0      TMA producer of A: A tile [128 x 128 B] into a STAGES-deep ring guarded by
-//               full/empty mbarriers (for a pair, both CTAs' loads count on the leader's full
-//               barrier); it also arms each stage's expected bytes.
+//   warp 0      TMA producers of A (lanes 0 and 16: even and odd K blocks): A tile [128 x
+//               128 B] into a STAGES-deep ring guarded by full/empty mbarriers (for a pair, both
+//               CTAs' loads count on the leader's full barrier); they arm each stage's bytes.
 //   warp 1      TMEM allocator and (leader only) the single thread that issues tcgen05.mma
 //               kind::f8f6f4, four K=32 steps per K block, into one of 512/BN TMEM buffers, and
 //               commits the stage (empty) and the buffer (tfull) — to both CTAs of a pair.
-//   warp 2      loads B (and, for contiguous pair tiles, first lists the pairs once).
-//   warp 3      loads the A-scale ring.
+//   warp 2      loads B, lanes 0 and 16 as for A (and, for contiguous pair tiles, first lists
+//               the pairs once).
+//   warp 3      loads the A-scale ring (four threads, one per K block mod 4).
 //   warps 4-11  two math warpgroups. Warp w reads TMEM lanes 32·(w%4)..+31 (its 32 rows);
 //               warpgroup j owns columns [j·BN/2, (j+1)·BN/2). Per K block: wait for the TMEM
 //               buffer, load the partial in 32-column batches (the next batch in flight while
@@ -85,14 +86,14 @@ struct GemmLayout {
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_D = OFF_B + STAGES * B_BYTES;
-    // A-scale ring: one 128-float row per K block. The producer can run at most STAGES + NBUF
-    // K blocks ahead of the math warps, so STAGES + NBUF + 1 slots need no "empty" barrier.
+    // A-scale ring: one 128-float row per K block, with full/empty barriers of its own (its
+    // loads are not on the MMA's path, so the operand ring's barriers cannot pace them).
     static constexpr int SFS = STAGES + NBUF + 1;
     static constexpr int OFF_SFA = OFF_D + 8 * SLAB_BYTES;
     static constexpr int OFF_PAIRS = OFF_SFA + SFS * BM * 4;
     static constexpr int PAIR_BYTES = PAIR_LIST ? MAX_PAIR_BLOCKS * 2 : 0;
     static constexpr int OFF_BAR = OFF_PAIRS + PAIR_BYTES;
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 8 + SFS;
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 8 + 2 * SFS;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int BYTES = OFF_MISC + static_cast<int>(sizeof(WaitCtx)) + 16;
     static constexpr int ALLOC = BYTES + 1024;               // slack to align the base to 1024 B
@@ -255,6 +256,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint64_t *tempty = tfull + NBUF;
     uint64_t *cfull = tempty + NBUF;
     uint64_t *sfa_full = cfull + 8;
+    uint64_t *sfa_empty = sfa_full + L::SFS;
     const float *sfa_ring = reinterpret_cast<const float *>(smem + L::OFF_SFA);
     WaitCtx *ctx = reinterpret_cast<WaitCtx *>(smem + L::OFF_MISC);
     int *num_pairs_smem = reinterpret_cast<int *>(smem + L::OFF_MISC + sizeof(WaitCtx));
@@ -278,7 +280,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             mbar_init(&tempty[b], PAIR ? 16 : 8);
         }
         for (int w = 0; w < 8; ++w) mbar_init(&cfull[w], 1);
-        for (int j = 0; j < L::SFS; ++j) mbar_init(&sfa_full[j], 1);
+        for (int j = 0; j < L::SFS; ++j) {
+            mbar_init(&sfa_full[j], 1);
+            mbar_init(&sfa_empty[j], 8);   // one arrive per math warp
+        }
         ctx->abort = 0;
         ctx->err = p.err;
         ctx->limit_ns = p.timeout_ns;
@@ -327,28 +332,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
     if (warp < 4) {
         reg_dealloc<56>();
-        // TMA producers, one thread per stream: warp 0 arms each stage and loads A, warp 2 loads
-        // B, warp 3 loads the A scales. One thread's bulk copies are served one after another
-        // (a fixed cost per copy, whatever its size), so three streams keep three in flight.
-        // All three wait on the same "empty" barrier of the ring; none can run more than
-        // STAGES K blocks ahead of the others, since a stage is only freed once all its loads
-        // have landed and the MMA has consumed it.
-        const int stream = warp == 0 ? 0 : (warp == 2 ? 1 : (warp == 3 ? 2 : -1));
-        if (stream >= 0 && lane == 0) {
+        // TMA producers. One thread's bulk copies are served one after another (a fixed cost
+        // per copy, whatever its size), so A and B each get two threads (lanes 0 and 16 of warps
+        // 0 and 2: even and odd K blocks) and the small A-scale copies four (lanes 0, 8, 16, 24
+        // of warp 3: K block mod 4); the A thread of a K block arms its stage. All wait on the same "empty" barriers of the ring; none can run
+        // more than STAGES K blocks ahead of the others, since a stage is only freed once all
+        // its loads have landed and the MMA has consumed it.
+        const int stream = warp == 0 || warp == 2 ? ((lane & 15) == 0 ? warp >> 1 : -1) : (warp == 3 && (lane & 7) == 0 ? 2 : -1);
+        // A/B (weights/activations): K block parity = lane / 16; A scales: K block mod 4 = lane / 8
+        const uint32_t parity = static_cast<uint32_t>(stream == 2 ? lane >> 3 : lane >> 4);
+        const uint32_t nlanes = stream == 2 ? 4u : 2u;
+        if (stream >= 0) {
             uint32_t it = 0;
             for (int t = cid; t < num_tiles && !*abort_flag; t += ncid) {
                 const TileInfo ti = decode_tile<KIND, PAIR>(t, p, pair_first, num_pairs, rank);
                 if (!ti.valid) {
-                    if (stream == 0 && KIND == KIND_CONTIGUOUS && ti.g >= p.G) report_error(p.err, ERR_DATA);
+                    if (stream == 0 && parity == 0 && KIND == KIND_CONTIGUOUS && ti.g >= p.G) report_error(p.err, ERR_DATA);
                     continue;
                 }
                 const int brow = ti.n_blk * BN + static_cast<int>(rank) * L::B_ROWS;
                 for (int kb = 0; kb < p.Kb; ++kb, ++it) {
+                    if (it % nlanes != parity) continue;
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(&empty[s], ph ^ 1, ctx)) break;
                     if (stream == 2) {
                         const int j = it % L::SFS;
+                        if (!mbar_wait(&sfa_empty[j], ((it / L::SFS) & 1) ^ 1, ctx)) break;
                         float *sf = reinterpret_cast<float *>(smem + L::OFF_SFA) + j * BM;
                         mbar_arrive_expect_tx(&sfa_full[j], BM * 4);
                         if (KIND == KIND_MASKED)
@@ -357,6 +366,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                             tma_load_2d(&tm_sfa, &sfa_full[j], sf, ti.row0, kb);
                         continue;
                     }
+                    if (!mbar_wait(&empty[s], ph ^ 1, ctx)) break;
                     uint8_t *sa = smem + L::OFF_A + s * L::A_BYTES;
                     uint8_t *sb = smem + L::OFF_B + s * L::B_BYTES;
                     if (PAIR) {
@@ -472,6 +482,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 const float sa = sfa_ring[j * BM + q * 32 + lane];
                 tc_fence_after();
                 const float scale = sa * sb;
+                __syncwarp();
+                if (lane == 0) mbar_arrive_relaxed(&sfa_empty[j]);   // the slot is read
                 const float2 scale2 = make_float2(scale, scale);
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                        static_cast<uint32_t>(b * BN + wg * HALF);

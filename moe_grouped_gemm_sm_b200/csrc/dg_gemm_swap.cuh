@@ -1,5 +1,5 @@
-// dg_gemm_swap.cuh — FP8 block-scaled NT GEMM for few rows (decode): swapped operands and
-// split-K over a thread-block cluster, sm_100a.
+// dg_gemm_swap.cuh — FP8 block-scaled NT GEMM for few rows (decode): swapped operands and a
+// stream-K split of the work over every SM, sm_100a.
 //
 // Same result as dg_gemm.cuh, D = C + A·Bᵀ with per-128-K-block promotion (likun.im/craft/
 // deepgemm §一; aitangshan.cn/news/1491278 技术原理 §4), for layouts whose row count per group
@@ -10,15 +10,23 @@
 //     rows of a tile on the MMA's M side (TMEM lanes) and the TN activation rows on its N side
 //     (TMEM columns). A tile's 128 weight rows are one 128x128 scale block, so sfb is a single
 //     scalar per (tile, K block), and sfa becomes a per-column factor read from shared memory;
-//   * split-K: a cluster of S CTAs shares one tile, CTA r taking an even share of its K blocks;
-//     the S fp32 partials meet in distributed shared memory, where CTA r reduces rows
-//     [r·128/S, (r+1)·128/S) of the tile, adds C and writes D (bf16, round to nearest even).
-//     No global workspace is used and the reduction order is fixed (deterministic);
-//   * a deep TMA ring (6-8 stages of the 16 KB weight tile) keeps enough bytes in flight.
+//   * stream-K: the (tile, K block) units of all active tiles, in order, are cut into
+//     gridDim.x equal runs, one per CTA (one CTA per SM), so every SM streams the same number
+//     of weight bytes whatever the tile count. A CTA's run is a sequence of segments, each
+//     a range of K blocks of one tile. The CTA whose run holds a tile's first K block owns the
+//     tile: the other CTAs that cover part of it (higher-numbered, and for each of them it is
+//     the first segment of its run, done before anything else) leave fp32 partials in a
+//     global workspace, and the owner, for which the tile is the last segment of its run,
+//     adds them to its own in CTA order (a fixed order: results are deterministic), adds C and
+//     writes D (bf16, round to nearest even). Flags in the workspace tell the owner when a
+//     partial is complete; the owner clears each flag it consumed, so the workspace is back
+//     to all-zero flags at the end of every launch (CUDA-graph replays stay valid);
+//   * a deep TMA ring (5-8 stages of the 16 KB weight tile) keeps enough bytes in flight.
 //
-// CTA layout: warps 0, 2, 3 TMA producers (weights, activations, A scales), warp 1 TMEM
-// allocator + single-thread tcgen05.mma issuer (kind::f8f6f4, M = 128, N = TN), warps 4.. TN/64
-// math warpgroups (thread = weight row, registers = its warpgroup's 64 token columns).
+// CTA layout: warps 0, 2, 3 TMA producers (weights and activations on two threads each, the A
+// scales on four), warp 1 TMEM allocator + single-thread tcgen05.mma issuer (kind::f8f6f4,
+// M = 128, N = TN), warps 4.. TN/64 math warpgroups (thread = weight row, registers = its
+// warpgroup's 64 token columns).
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -29,19 +37,19 @@
 namespace dg {
 
 struct SwapParams {
-    int M;            // rows per group (dense: M <= TN; masked: M_max)
+    int M;            // rows per group (dense: M; masked: M_max)
     int N, K, G;
     int Kb, Nb;       // K/128, ceil(N/128)
     int ld_sfa;       // pad4(M)
     int n_tiles;      // ceil(N/128)
     int m_tiles;      // ceil(M/TN): token tiles per group
-    int num_tiles;    // (masked: G ·) m_tiles · n_tiles
-    int splits;       // S: CTAs per cluster along K
     int has_c;
     const float *sfb;
     const int32_t *masked_m;   // masked layout only
     const __nv_bfloat16 *c;
     __nv_bfloat16 *d;
+    float *ws;        // stream-K partials, [gridDim.x][TN][128] fp32
+    int *flags;       // [gridDim.x]; all zero between launches
     int *err;
     uint64_t timeout_ns;
 };
@@ -56,22 +64,88 @@ struct SwapLayout {
     static constexpr int X_BYTES = TN * BK;                  // activation tile: TN rows x 128 B
     static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
     static constexpr int NBUF = (512 / TN) > 4 ? 4 : (512 / TN);
-    static constexpr int SFS = STAGES + NBUF + 1;            // A-scale ring (see dg_gemm.cuh)
-    static constexpr int RED_BYTES = TN * 128 * 4;           // fp32 partial [TN][128], reuses the ring
+    static constexpr int SFS = STAGES + NBUF + 1;            // A-scale ring, own full/empty barriers
     static constexpr int OFF_W = 0;
     static constexpr int OFF_X = OFF_W + STAGES * W_BYTES;
     static constexpr int OFF_SFA = OFF_X + STAGES * X_BYTES;
-    static constexpr int OFF_C = OFF_SFA + SFS * TN * 4;        // C tile [TN][128] bf16 (S == 1 epilogue)
+    static constexpr int OFF_C = OFF_SFA + SFS * TN * 4;        // C tile [TN][128] bf16 (tile owner)
     static constexpr int C_BYTES = TN * 128 * 2;
     static constexpr int OFF_BAR = OFF_C + C_BYTES;
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + SFS + 1;
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 2 * SFS + 2;
+    static constexpr int PART_BYTES = TN * 128 * 4;          // one fp32 partial of a tile
+    static constexpr int MAX_PARTS = STAGES * STAGE_BYTES / PART_BYTES;   // fit the idle ring
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int BYTES = OFF_MISC + static_cast<int>(sizeof(WaitCtx));
     static constexpr int ALLOC = BYTES + 1024;
     static constexpr uint32_t TMEM_COLS = NBUF * TN <= 256 ? (NBUF * TN <= 128 ? 128 : 256) : 512;
     static_assert(OFF_X % 1024 == 0 && OFF_SFA % 16 == 0 && OFF_C % 128 == 0, "aligned tiles");
-    static_assert(STAGES * STAGE_BYTES >= RED_BYTES, "the reduction buffer reuses the operand ring");
     static_assert(ALLOC <= 232448, "shared memory budget");
+};
+
+// The active tiles, in the order the stream-K units run through them: for each group g, its
+// token tiles mt < ceil(rows_g / TN) (rows_g = M, or masked_m[g] clamped to [0, M]), and for
+// each token tile the weight tiles nt, nt fastest (consecutive tiles share the activations).
+template <int TN, int KIND>
+struct SwapTiles {
+    const SwapParams &p;
+    int count;
+    __device__ explicit SwapTiles(const SwapParams &pp) : p(pp) {
+        if (KIND == KIND_MASKED) {
+            count = 0;
+            for (int g = 0; g < p.G; ++g) count += (rows_of(g) + TN - 1) / TN * p.n_tiles;
+        } else {
+            count = p.m_tiles * p.n_tiles;
+        }
+    }
+    __device__ int rows_of(int g) const {
+        if (KIND != KIND_MASKED) return p.M;
+        const int mm = __ldg(p.masked_m + g);
+        return mm < 0 ? 0 : (mm > p.M ? p.M : mm);
+    }
+    // tile a -> group g, first token row m0, first weight row n0; returns the token rows of the
+    // tile that exist (>= 1 for a < count)
+    __device__ int coords(int a, int &g, int &m0, int &n0) const {
+        g = 0;
+        if (KIND == KIND_MASKED) {
+            while (g < p.G - 1) {
+                const int cnt = (rows_of(g) + TN - 1) / TN * p.n_tiles;
+                if (a < cnt) break;
+                a -= cnt;
+                ++g;
+            }
+        }
+        n0 = (a % p.n_tiles) * 128;
+        m0 = (a / p.n_tiles) * TN;
+        return min(TN, rows_of(g) - m0);
+    }
+};
+
+// A CTA's run of units [u0, u1) out of U = tiles · Kb (unit u = K block u % Kb of tile u / Kb);
+// the CTA holding unit u is cta_of(u). The units are cut over the first P CTAs of the grid
+// (the others get empty runs), P small enough that every run holds at least
+// ceil((Kb - 1) / max_parts) units: then no tile is spread over more than max_parts + 1 runs,
+// i.e. no owner has more than max_parts partials to add (and no run is empty, which the
+// masked layout, with fewer units than the grid was sized for, would otherwise allow). Runs
+// are walked segment by segment: segment() gives the tile and the K-block range
+// [kb_begin, kb_end) of the segment starting at unit u.
+struct StreamK {
+    long long U, u0, u1;
+    int Kb, P;
+    __device__ StreamK(int tiles, int kb, int c, int grid, int max_parts) : Kb(kb) {
+        U = static_cast<long long>(tiles) * kb;
+        const long long min_run = kb > 1 ? (kb - 1 + max_parts - 1) / max_parts : 1;
+        const long long pmax = U / min_run > 1 ? U / min_run : 1;
+        P = pmax < grid ? static_cast<int>(pmax) : grid;
+        u0 = c < P ? U * c / P : U;
+        u1 = c < P ? U * (c + 1) / P : U;
+    }
+    __device__ int cta_of(long long u) const { return static_cast<int>(((u + 1) * P - 1) / U); }
+    __device__ void segment(long long u, int &tile, int &kb_begin, int &kb_end) const {
+        tile = static_cast<int>(u / Kb);
+        kb_begin = static_cast<int>(u - static_cast<long long>(tile) * Kb);
+        const long long rest = u1 - u;
+        kb_end = rest < Kb - kb_begin ? kb_begin + static_cast<int>(rest) : Kb;
+    }
 };
 
 template <int TN, int STAGES, int KIND>
@@ -90,47 +164,19 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + NBUF;
     uint64_t *sfa_full = tempty + NBUF;
-    uint64_t *c_full = sfa_full + L::SFS;
+    uint64_t *sfa_empty = sfa_full + L::SFS;
+    uint64_t *c_full = sfa_empty + L::SFS;
+    uint64_t *fix_full = c_full + 1;
     const __nv_bfloat16 *c_tile = reinterpret_cast<const __nv_bfloat16 *>(smem + L::OFF_C);
     WaitCtx *ctx = reinterpret_cast<WaitCtx *>(smem + L::OFF_MISC);
     const float *sfa_ring = reinterpret_cast<const float *>(smem + L::OFF_SFA);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int S = p.splits;
-    const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
-    // S == 1: persistent CTAs stride over the tiles; S > 1: one tile per cluster (grid = tiles·S)
-    const int cid = S > 1 ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
-    const int ncid = S > 1 ? p.num_tiles : static_cast<int>(gridDim.x);
-    const int per = (p.Kb + S - 1) / S;                      // K blocks per split
-    const int kb0 = static_cast<int>(rank) * per;
-    const int kb1 = min(p.Kb, kb0 + per);
-    const int nkb = max(0, kb1 - kb0);
-
-    // tile t = (g · m_tiles + mt) · n_tiles + nt: weight tile nt of expert g, token tile mt;
-    // returns the number of token rows of the tile that exist (<= 0: nothing to do)
-    auto tile_rows = [&](int t, int &g, int &m0, int &n0) {
-        const int nt = t % p.n_tiles;
-        const int mt = (t / p.n_tiles) % p.m_tiles;
-        g = KIND == KIND_MASKED ? t / (p.n_tiles * p.m_tiles) : 0;
-        n0 = nt * 128;
-        m0 = mt * TN;
-        int valid = p.M;
-        if (KIND == KIND_MASKED) {
-            const int mm = __ldg(p.masked_m + g);
-            valid = mm < 0 ? 0 : (mm > p.M ? p.M : mm);
-        }
-        return min(TN, valid - m0);
-    };
     if (KIND == KIND_MASKED && blockIdx.x == 0 && threadIdx.x == 0) {
         for (int gg = 0; gg < p.G; ++gg)
             if (__ldg(p.masked_m + gg) > p.M) report_error(p.err, ERR_DATA);
     }
-    if (S > 1) {                                           // every CTA of the cluster agrees
-        int g_, m0_, n0_;
-        if (tile_rows(cid, g_, m0_, n0_) <= 0) return;
-    }
-
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -140,8 +186,12 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 4 * L::NWG);
         }
-        for (int j = 0; j < L::SFS; ++j) mbar_init(&sfa_full[j], 1);
+        for (int j = 0; j < L::SFS; ++j) {
+            mbar_init(&sfa_full[j], 1);
+            mbar_init(&sfa_empty[j], 4 * L::NWG);   // one arrive per math warp
+        }
         mbar_init(c_full, 1);
+        mbar_init(fix_full, 1);
         ctx->abort = 0;
         ctx->err = p.err;
         ctx->limit_ns = p.timeout_ns;
@@ -162,39 +212,50 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = ctx->tmem_base;
     volatile int *abort_flag = &ctx->abort;
-
-    float acc[COLS];
-    int g = 0, m0 = 0, n0 = 0, rows = 0;                   // the last tile (split reduction)
+    const SwapTiles<TN, KIND> tiles(p);
+    const StreamK sk(tiles.count, p.Kb, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x), L::MAX_PARTS);
 
     if (warp < 4) {
-        // TMA producers, one thread per stream (one thread's bulk copies are served one after
-        // another): warp 0 arms each stage and loads the weights, warp 2 the activations,
-        // warp 3 the A scales. All wait on the ring's "empty" barriers.
-        const int stream = warp == 0 ? 0 : (warp == 2 ? 1 : (warp == 3 ? 2 : -1));
-        if (stream >= 0 && lane == 0) {
+        // TMA producers. One thread's bulk copies are served one after another, so the weights
+        // and the activations each get two threads (lanes 0 and 16 of warps 0 and 2, even and
+        // odd K blocks) and the small A-scale copies four (lanes 0, 8, 16, 24 of warp 3, K block
+        // mod 4). The weight thread of a K block arms its stage. All wait on the ring's "empty"
+        // barriers.
+        const int stream = warp == 0 || warp == 2 ? ((lane & 15) == 0 ? warp >> 1 : -1) : (warp == 3 && (lane & 7) == 0 ? 2 : -1);
+        // A/B (weights/activations): K block parity = lane / 16; A scales: K block mod 4 = lane / 8
+        const uint32_t parity = static_cast<uint32_t>(stream == 2 ? lane >> 3 : lane >> 4);
+        const uint32_t nlanes = stream == 2 ? 4u : 2u;
+        if (stream >= 0) {
+            // the weights are read once: evict them first; activations and A scales are read
+            // again by the CTAs working on other weight tiles: keep them
+            const uint64_t pol = stream == 0 ? l2_policy_evict_first() : l2_policy_evict_last();
             uint32_t it = 0;
-            for (int t = cid; t < p.num_tiles && !*abort_flag; t += ncid) {
-                int tg, tm0, tn0;
-                if (tile_rows(t, tg, tm0, tn0) <= 0) continue;
-                for (int i = 0; i < nkb; ++i, ++it) {
-                    const int kb = kb0 + i;
+            for (long long u = sk.u0; u < sk.u1 && !*abort_flag;) {
+                int tile, kbs, kbe, tg, tm0, tn0;
+                sk.segment(u, tile, kbs, kbe);
+                u += kbe - kbs;
+                tiles.coords(tile, tg, tm0, tn0);
+                for (int kb = kbs; kb < kbe; ++kb, ++it) {
+                    if (it % nlanes != parity) continue;
                     const int s = it % STAGES;
-                    if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, ctx)) break;
+                    const int j = it % L::SFS;
+                    if (!mbar_wait(stream == 2 ? &sfa_empty[j] : &empty[s],
+                                   stream == 2 ? ((it / L::SFS) & 1) ^ 1 : ((it / STAGES) & 1) ^ 1, ctx))
+                        break;
                     if (stream == 2) {
-                        const int j = it % L::SFS;
                         mbar_arrive_expect_tx(&sfa_full[j], TN * 4);
                         float *sf = reinterpret_cast<float *>(smem + L::OFF_SFA) + j * TN;
                         if (KIND == KIND_MASKED)
-                            tma_load_3d(&tm_sfa, &sfa_full[j], sf, tm0, kb, tg);
+                            tma_load_3d_hint(&tm_sfa, &sfa_full[j], sf, tm0, kb, tg, pol);
                         else
-                            tma_load_2d(&tm_sfa, &sfa_full[j], sf, tm0, kb);
+                            tma_load_2d_hint(&tm_sfa, &sfa_full[j], sf, tm0, kb, pol);
                     } else if (stream == 0) {
                         mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
-                        tma_load_3d(&tm_w, &full[s], smem + L::OFF_W + s * L::W_BYTES, kb * BK, tn0, tg);
+                        tma_load_3d_hint(&tm_w, &full[s], smem + L::OFF_W + s * L::W_BYTES, kb * BK, tn0, tg, pol);
                     } else if (KIND == KIND_MASKED) {
-                        tma_load_3d(&tm_x, &full[s], smem + L::OFF_X + s * L::X_BYTES, kb * BK, tm0, tg);
+                        tma_load_3d_hint(&tm_x, &full[s], smem + L::OFF_X + s * L::X_BYTES, kb * BK, tm0, tg, pol);
                     } else {
-                        tma_load_2d(&tm_x, &full[s], smem + L::OFF_X + s * L::X_BYTES, kb * BK, tm0);
+                        tma_load_2d_hint(&tm_x, &full[s], smem + L::OFF_X + s * L::X_BYTES, kb * BK, tm0, pol);
                     }
                 }
             }
@@ -202,10 +263,11 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
             // ---------------- MMA issuer ----------------
             constexpr uint32_t IDESC = idesc_f8_e4m3_f32<128, TN>();
             uint32_t it = 0;
-            for (int t = cid; t < p.num_tiles && !*abort_flag; t += ncid) {
-                int tg, tm0, tn0;
-                if (tile_rows(t, tg, tm0, tn0) <= 0) continue;
-                for (int i = 0; i < nkb; ++i, ++it) {
+            for (long long u = sk.u0; u < sk.u1 && !*abort_flag;) {
+                int tile, kbs, kbe;
+                sk.segment(u, tile, kbs, kbe);
+                u += kbe - kbs;
+                for (int kb = kbs; kb < kbe; ++kb, ++it) {
                     const int s = it % STAGES;
                     const int b = it % NBUF;
                     if (!mbar_wait(&full[s], (it / STAGES) & 1, ctx)) break;
@@ -222,21 +284,28 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
             }
         }
     } else {
-        // ---------------- math warpgroups: promotion (+ the epilogue when S == 1) ----------------
+        // ---------------- math warpgroups: promotion, partials, tile epilogue ----------------
+        // Every math thread walks the same segments and meets the same named barriers, even
+        // after a wait has given up (then the work is skipped), so no barrier is left waiting.
         const int wg = (warp - 4) >> 2;                    // token columns [wg·64, wg·64 + 64)
         const int q = warp & 3;                            // TMEM lane quadrant = weight rows 32q..
         const int n = q * 32 + lane;                       // this thread's weight row in the tile
+        const int c_self = static_cast<int>(blockIdx.x);
         uint32_t it = 0, ctile = 0;
         bool ok = true;
-        for (int t = cid; t < p.num_tiles && ok; t += ncid) {
-            rows = tile_rows(t, g, m0, n0);
-            if (rows <= 0) continue;
+        float acc[COLS];
+        for (long long u = sk.u0; u < sk.u1;) {
+            int tile, kbs, kbe, g, m0, n0;
+            sk.segment(u, tile, kbs, kbe);
+            u += kbe - kbs;
+            const int rows = tiles.coords(tile, g, m0, n0);
+            const bool owner = kbs == 0;                   // this CTA holds the tile's first K block
             const int nt = n0 / 128;
-            const bool do_c = S == 1 && p.has_c;
+            const bool do_c = owner && p.has_c;
             if (do_c) {
                 // the previous tile's C has been read by every math thread before it is replaced
                 asm volatile("bar.sync 1, %0;" ::"n"(128 * L::NWG) : "memory");
-                if (threadIdx.x == 128) {
+                if (threadIdx.x == 128 && ok) {
                     fence_proxy_async_smem();
                     mbar_arrive_expect_tx(c_full, L::C_BYTES);
                     if (KIND == KIND_MASKED)
@@ -248,20 +317,20 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
 #pragma unroll
             for (int i = 0; i < COLS; ++i) acc[i] = 0.f;
             const float *sfb_col = p.sfb + (static_cast<size_t>(g) * p.Nb + nt) * p.Kb;
-            float sb_win = kb0 + lane < kb1 ? __ldg(sfb_col + kb0 + lane) : 0.f;
-            float sb_nxt = kb0 + 32 + lane < kb1 ? __ldg(sfb_col + kb0 + 32 + lane) : 0.f;
-            for (int i = 0; i < nkb; ++i, ++it) {
+            float sb_win = kbs + lane < kbe ? __ldg(sfb_col + kbs + lane) : 0.f;
+            float sb_nxt = kbs + 32 + lane < kbe ? __ldg(sfb_col + kbs + 32 + lane) : 0.f;
+            for (int i = 0; i < kbe - kbs; ++i, ++it) {
                 const int b = it % NBUF;
                 const int j = it % L::SFS;
                 if ((i & 31) == 0 && i > 0) {
                     sb_win = sb_nxt;
-                    sb_nxt = kb0 + i + 32 + lane < kb1 ? __ldg(sfb_col + kb0 + i + 32 + lane) : 0.f;
+                    sb_nxt = kbs + i + 32 + lane < kbe ? __ldg(sfb_col + kbs + i + 32 + lane) : 0.f;
                 }
                 const float sb = __shfl_sync(0xFFFFFFFFu, sb_win, i & 31);
+                if (!ok) continue;
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], (it / NBUF) & 1, ctx));
-                if (!ok) break;
-                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sfa_full[j], (it / L::SFS) & 1, ctx));
-                if (!ok) break;
+                if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sfa_full[j], (it / L::SFS) & 1, ctx));
+                if (!ok) continue;
                 tc_fence_after();
                 const float *sfa_row = sfa_ring + j * TN + wg * COLS;
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
@@ -294,113 +363,91 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_relaxed(&tempty[b]);
-            }
-            if (!ok) break;
-            if (S == 1) {
-                if (do_c) {
-                    ok = __all_sync(0xFFFFFFFFu, mbar_wait(c_full, ctile & 1, ctx));
-                    ++ctile;
-                    if (!ok) break;
+                if (lane == 0) {
+                    mbar_arrive_relaxed(&sfa_empty[j]);
+                    mbar_arrive_relaxed(&tempty[b]);
                 }
-                // direct epilogue: D[g][m0+m][n0+n] for the tile's token rows; a warp stores 32
-                // consecutive columns of one token row per instruction; C comes from the tile
-                // TMA prefetched at tile start ([m][n] in shared memory: conflict-free reads)
-                if (n0 + n < p.N) {
-                    const size_t base = (static_cast<size_t>(g) * p.M + m0) * p.N + n0 + n;
+            }
+            if (!owner) {
+                // a partial (always this CTA's first segment): [TN token rows][128 weight rows] fp32,
+                // published to the owner by the CTA's flag once every math thread's stores are
+                // ordered before it (gpu-scope fence, then a barrier of the math threads)
+                float *ws_self = p.ws + static_cast<size_t>(c_self) * TN * 128;
+                if (ok) {
 #pragma unroll
-                    for (int e = 0; e < COLS; ++e) {
-                        const int m = wg * COLS + e;
-                        if (m < rows) {
-                            const float cv = do_c ? __bfloat162float(c_tile[m * 128 + n]) : 0.f;
-                            p.d[base + static_cast<size_t>(m) * p.N] = __float2bfloat16_rn(acc[e] + cv);
+                    for (int e = 0; e < COLS; ++e) __stcg(ws_self + (wg * COLS + e) * 128 + n, acc[e]);
+                    __threadfence();
+                }
+                ok = named_barrier_and(2, 128 * L::NWG, ok);
+                if (threadIdx.x == 128 && ok) flag_store_release(p.flags + c_self, 1);
+                continue;
+            }
+            if (kbe < p.Kb) {
+                // The tile's later K blocks are partials of CTAs c_self+1 .. j1 (at most
+                // MAX_PARTS). Their flags are waited for (and cleared for the next launch), the
+                // partials copied in bulk into the operand ring, idle now (this is the run's last
+                // segment and its MMAs are done), and added in CTA order.
+                const int j1 = sk.cta_of(static_cast<long long>(tile) * p.Kb + p.Kb - 1);
+                const int nparts = j1 - c_self;
+                bool got = ok && nparts <= L::MAX_PARTS;
+                if (threadIdx.x == 128 && ok && !got) report_error(ctx->err, ERR_DATA);
+                if (threadIdx.x == 128 && got) {
+                    const uint64_t t0 = globaltimer_ns();
+                    for (int jj = c_self + 1; jj <= j1 && got; ++jj) {
+                        while (flag_load_acquire(p.flags + jj) == 0) {
+                            if (*abort_flag) {
+                                got = false;
+                                break;
+                            }
+                            if (globaltimer_ns() - t0 > ctx->limit_ns) {
+                                report_error(ctx->err, ERR_TIMEOUT);
+                                *abort_flag = 1;
+                                got = false;
+                                break;
+                            }
                         }
+                        if (got) p.flags[jj] = 0;
+                    }
+                    if (got) mbar_arrive_expect_tx(fix_full, static_cast<uint32_t>(nparts) * L::PART_BYTES);
+                }
+                ok = named_barrier_and(2, 128 * L::NWG, got);
+                float *parts = reinterpret_cast<float *>(smem + L::OFF_W);
+                if (ok && warp == 4 && lane < nparts) {   // one bulk copy per lane, all in flight
+                    fence_proxy_async_global();
+                    bulk_load(parts + static_cast<size_t>(lane) * TN * 128,
+                              p.ws + static_cast<size_t>(c_self + 1 + lane) * TN * 128, L::PART_BYTES, fix_full);
+                }
+                if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(fix_full, 0, ctx));
+                if (ok) {
+                    for (int k = 0; k < nparts; ++k) {
+#pragma unroll
+                        for (int e = 0; e < COLS; ++e) acc[e] += parts[(k * TN + wg * COLS + e) * 128 + n];
+                    }
+                }
+            }
+            if (do_c && ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(c_full, ctile & 1, ctx));
+            if (do_c) ++ctile;
+            if (!ok) continue;
+            // tile epilogue: D[g][m0+m][n0+n] for the tile's token rows; a warp stores 32
+            // consecutive columns of one token row per instruction; C comes from the tile TMA
+            // loaded at the segment's start ([m][n] in shared memory: conflict-free reads)
+            if (n0 + n < p.N) {
+                const size_t base = (static_cast<size_t>(g) * p.M + m0) * p.N + n0 + n;
+#pragma unroll
+                for (int e = 0; e < COLS; ++e) {
+                    const int m = wg * COLS + e;
+                    if (m < rows) {
+                        const float cv = do_c ? __bfloat162float(c_tile[m * 128 + n]) : 0.f;
+                        p.d[base + static_cast<size_t>(m) * p.N] = __float2bfloat16_rn(acc[e] + cv);
                     }
                 }
             }
         }
     }
 
-    if (S > 1) {
-        // ---------------- split-K reduction through distributed shared memory ----------------
-        // The cluster's one tile is done: the operand ring is reused for this CTA's fp32 partial,
-        // laid out [TN token rows][128 weight rows] (each math thread owns one weight row).
-        __syncwarp();
-        tc_fence_before();
-        __syncthreads();
-        float *red = reinterpret_cast<float *>(smem + L::OFF_W);
-        if (warp >= 4) {
-            const int n = (warp & 3) * 32 + lane;
-            const int wg = (warp - 4) >> 2;
-#pragma unroll
-            for (int i = 0; i < COLS; ++i) red[(wg * COLS + i) * 128 + n] = acc[i];
-        }
-        __syncwarp();
-        cluster_sync();
-        int g_, m0_, n0_;
-        const int trows = tile_rows(cid, g_, m0_, n0_);
-        // CTA `rank` owns weight rows [rank·R, rank·R + R) of the tile, R = 128/S: a thread sums
-        // groups of 4 consecutive weight rows of one token row over the S partials; all loads
-        // of a thread (up to 4 items) are issued before any is used.
-        const int R = 128 / S;
-        const int groups = R / 4;
-        const int items = trows * groups;
-        const uint32_t red_local = smem_u32(red);
-        for (int base_it = 0; base_it < items; base_it += 4 * static_cast<int>(blockDim.x)) {
-            float4 sum[4];
-            float4 cvals[4];
-            bool live[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int itm = base_it + u * static_cast<int>(blockDim.x) + static_cast<int>(threadIdx.x);
-                live[u] = itm < items;
-                sum[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                cvals[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (!live[u]) continue;
-                const int m = itm / groups;
-                const int nn = static_cast<int>(rank) * R + (itm % groups) * 4;
-                const uint32_t off = static_cast<uint32_t>((m * 128 + nn) * 4);
-                for (int src = 0; src < S; ++src) {
-                    const float4 v = ld_shared_cluster_v4(mapa_shared(red_local + off, src));
-                    sum[u].x += v.x;
-                    sum[u].y += v.y;
-                    sum[u].z += v.z;
-                    sum[u].w += v.w;
-                }
-                const int col = n0_ + nn;
-                if (p.has_c && col < p.N) {
-                    const size_t o = (static_cast<size_t>(g_) * p.M + m0_ + m) * p.N + col;
-                    const uint2 cv = *reinterpret_cast<const uint2 *>(p.c + o);
-                    const __nv_bfloat162 c01 = *reinterpret_cast<const __nv_bfloat162 *>(&cv.x);
-                    const __nv_bfloat162 c23 = *reinterpret_cast<const __nv_bfloat162 *>(&cv.y);
-                    cvals[u] = make_float4(__bfloat162float(c01.x), __bfloat162float(c01.y), __bfloat162float(c23.x),
-                                           __bfloat162float(c23.y));
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (!live[u]) continue;
-                const int itm = base_it + u * static_cast<int>(blockDim.x) + static_cast<int>(threadIdx.x);
-                const int m = itm / groups;
-                const int nn = static_cast<int>(rank) * R + (itm % groups) * 4;
-                const int col = n0_ + nn;
-                if (col >= p.N) continue;                      // N % 8 == 0: a group of 4 is in or out
-                const size_t o = (static_cast<size_t>(g_) * p.M + m0_ + m) * p.N + col;
-                __nv_bfloat162 h01 = __floats2bfloat162_rn(sum[u].x + cvals[u].x, sum[u].y + cvals[u].y);
-                __nv_bfloat162 h23 = __floats2bfloat162_rn(sum[u].z + cvals[u].z, sum[u].w + cvals[u].w);
-                uint2 w;
-                w.x = *reinterpret_cast<uint32_t *>(&h01);
-                w.y = *reinterpret_cast<uint32_t *>(&h23);
-                *reinterpret_cast<uint2 *>(p.d + o) = w;
-            }
-        }
-        __syncwarp();                                      // lanes left the loop at different trips
-        cluster_sync();                                    // peers may still read this CTA's partial
-    } else {
-        __syncwarp();
-        tc_fence_before();
-        __syncthreads();
-    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
