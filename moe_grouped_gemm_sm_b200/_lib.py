@@ -48,6 +48,7 @@ def load():
         P, I = ctypes.c_void_p, ctypes.c_int
         sig = {
             "dg_fp8_gemm_nt": [P, P, P, P, P, P, I, I, I, P],
+            "dg_fp8_gemm_nt_noalloc": [P, P, P, P, P, P, I, I, I, P],
             "dg_m_grouped_fp8_gemm_nt_contiguous": [P, P, P, P, P, P, P, I, I, I, I, P],
             "dg_m_grouped_fp8_gemm_nt_masked": [P, P, P, P, P, P, P, I, I, I, I, I, P],
             "dg_transform_sf": [P, P, I, I, I, P],
@@ -90,6 +91,11 @@ def _call(name, *args):
 
 def dg_fp8_gemm_nt(a, sfa, b, sfb, c, d, M, N, K, stream=None):
     _call("dg_fp8_gemm_nt", _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(c), _ptr(d), M, N, K, _stream(stream))
+
+
+def dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, c, d, M, N, K, stream=None):
+    _call("dg_fp8_gemm_nt_noalloc", _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(c), _ptr(d), M, N, K,
+          _stream(stream))
 
 
 def dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, c, d, grouped_layout, M_sum, N, K, G, stream=None):

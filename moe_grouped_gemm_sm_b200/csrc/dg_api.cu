@@ -22,11 +22,19 @@ constexpr int kMaxDevices = 64;
 
 __device__ int g_device_error;   // see dg_get_device_error()
 
+// Scratch of dg_fp8_gemm_nt_noalloc: the few-row kernel's stream-K partials and flags for up to
+// kStaticSlots CTAs, in the module's own device memory (zero-initialised at load).
+constexpr int kStaticSlots = 256;
+static __device__ __align__(256) float g_static_ws[kStaticSlots * 128 * 128];
+static __device__ __align__(256) int g_static_flags[kStaticSlots];
+
 struct DeviceInfo {
     bool ready = false;
     int sm_count = 0;
     int cc_major = 0, cc_minor = 0;
     int *err = nullptr;          // device address of g_device_error
+    float *static_ws = nullptr;  // device addresses of g_static_ws and g_static_flags
+    int *static_flags = nullptr;
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -46,7 +54,10 @@ dg_status device_info(const DeviceInfo **out) {
             if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DG_ERR_CUDA;
             cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
             cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
-            if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_device_error) != cudaSuccess) return DG_ERR_CUDA;
+            if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_device_error) != cudaSuccess ||
+                cudaGetSymbolAddress(reinterpret_cast<void **>(&d.static_ws), g_static_ws) != cudaSuccess ||
+                cudaGetSymbolAddress(reinterpret_cast<void **>(&d.static_flags), g_static_flags) != cudaSuccess)
+                return DG_ERR_CUDA;
             if (!g_encode) {
                 cudaDriverEntryPointQueryResult q;
                 void *fn = nullptr;
@@ -372,10 +383,11 @@ bool swap_workspace(int dev, int sm_count, cudaStream_t st, SwapWorkspace *out) 
 }
 
 // After a device error a launch may have stopped with flags still set: zero this device's.
-void reset_swap_flags(int dev) {
+void reset_swap_flags(int dev, const DeviceInfo *di) {
     std::lock_guard<std::mutex> lk(g_mu);
     for (const SwapWorkspace &w : g_swap_ws)
         if (w.dev == dev) cudaMemset(w.flags, 0, static_cast<size_t>(w.slots) * sizeof(int));
+    cudaMemset(di->static_flags, 0, kStaticSlots * sizeof(int));
 }
 
 template <int TN, int STAGES, int KIND>
@@ -403,17 +415,11 @@ dg_status launch_swap(const SwapMaps &mp, const dg::SwapParams &p, long long til
     return from_cuda(cudaGetLastError());
 }
 
-// Returns DG_ERR_UNSUPPORTED (nothing launched) when no workspace is available for `st`.
+// The few-row GEMM with the given stream-K scratch (partials for >= sm_count slots, flags zero).
 template <int KIND>
-dg_status run_swap(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
-                   const int32_t *masked_m, int expected_m, int rows, int N, int K, int G, cudaStream_t st) {
-    const DeviceInfo *di = nullptr;
-    dg_status s = device_info(&di);
-    if (s != DG_OK) return s;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
-    SwapWorkspace w;
-    if (!swap_workspace(dev, di->sm_count, st, &w)) return DG_ERR_UNSUPPORTED;
+dg_status run_swap_with(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
+                        const int32_t *masked_m, int expected_m, int rows, int N, int K, int G, cudaStream_t st,
+                        const DeviceInfo *di, float *ws, int *flags) {
     const bool batched = KIND == dg::KIND_MASKED;
     const int hint = batched ? (expected_m > 0 ? expected_m : rows) : rows;
     const int tn = hint <= 64 ? 64 : 128;
@@ -432,8 +438,8 @@ dg_status run_swap(const void *a, const float *sfa, const void *b, const float *
     p.masked_m = masked_m;
     p.c = static_cast<const __nv_bfloat16 *>(c);
     p.d = static_cast<__nv_bfloat16 *>(d);
-    p.ws = w.ws;
-    p.flags = w.flags;
+    p.ws = ws;
+    p.flags = flags;
     p.err = di->err;
     p.timeout_ns = wait_limit_ns();
     // the largest possible tile set: masked groups may use fewer
@@ -442,6 +448,21 @@ dg_status run_swap(const void *a, const float *sfa, const void *b, const float *
     if (!build_swap_maps(mp, a, sfa, b, c, rows, N, K, G, tn, batched)) return DG_ERR_INVALID_ARG;
     if (tn == 64) return launch_swap<64, 8, KIND>(mp, p, tiles, di, st);
     return launch_swap<128, 5, KIND>(mp, p, tiles, di, st);
+}
+
+// The few-row GEMM with the per-stream workspace. Returns DG_ERR_UNSUPPORTED (nothing
+// launched) when no workspace is available for `st`.
+template <int KIND>
+dg_status run_swap(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
+                   const int32_t *masked_m, int expected_m, int rows, int N, int K, int G, cudaStream_t st) {
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
+    SwapWorkspace w;
+    if (!swap_workspace(dev, di->sm_count, st, &w)) return DG_ERR_UNSUPPORTED;
+    return run_swap_with<KIND>(a, sfa, b, sfb, c, d, masked_m, expected_m, rows, N, K, G, st, di, w.ws, w.flags);
 }
 
 dg_status check_gemm_common(const void *a, const float *sfa, const void *b, const float *sfb, const void *c,
@@ -472,6 +493,21 @@ dg_status dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const f
     }
     return run_gemm<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, nullptr, M, N, K, 1,
                                     static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b, const float *sfb, const void *c,
+                                 void *d, int M, int N, int K, void *stream) {
+    if (M < 0) return DG_ERR_INVALID_ARG;
+    dg_status s = check_gemm_common(a, sfa, b, sfb, c, d, N, K);
+    if (s != DG_OK) return s;
+    if (M > 128) return DG_ERR_UNSUPPORTED;
+    if (M == 0) return DG_OK;
+    const DeviceInfo *di = nullptr;
+    s = device_info(&di);
+    if (s != DG_OK) return s;
+    if (di->sm_count > kStaticSlots) return DG_ERR_UNSUPPORTED;
+    return run_swap_with<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, 0, M, N, K, 1,
+                                         static_cast<cudaStream_t>(stream), di, di->static_ws, di->static_flags);
 }
 
 dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
@@ -566,7 +602,7 @@ dg_status dg_get_device_error(void *stream) {
         const int zero = 0;
         if (cudaMemcpy(di->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return DG_ERR_CUDA;
         int dev = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess) reset_swap_flags(dev);
+        if (cudaGetDevice(&dev) == cudaSuccess) reset_swap_flags(dev, di);
     }
     if (v == dg::ERR_TIMEOUT) return DG_ERR_TIMEOUT;
     if (v != 0) return DG_ERR_DEVICE;
