@@ -153,7 +153,7 @@ struct GemmMaps {
 // Operand maps of one GEMM call. rows = rows of A/C/D per group; b_rows = rows of B one CTA
 // loads; batched = 3D maps over G groups for A, C and D (masked layout).
 bool build_maps(GemmMaps &mp, const void *a, const float *sfa, const void *b, const void *c, void *d, int rows, int N,
-                int K, int G, int b_rows, bool batched) {
+                int K, int G, int b_rows, bool batched, int slab_blocks) {
     const uint64_t Gg = static_cast<uint64_t>(G);
     {   // sfa: fp32 [G?][Kb][pad4(rows)], box 128 x 1 (one K block's scales of a 128-row block)
         const uint64_t Kb = static_cast<uint64_t>(K / 128), ld = static_cast<uint64_t>(pad4(rows));
@@ -178,6 +178,22 @@ bool build_maps(GemmMaps &mp, const void *a, const float *sfa, const void *b, co
         const uint32_t box[3] = {128, static_cast<uint32_t>(b_rows), 1};
         if (!encode(&mp.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return false;
+    }
+    if (slab_blocks > 0) {
+        // C, D: bf16 [rows][N] seen as {64 columns, rows, N/64 column blocks}, box 64 x 32 x
+        // slab_blocks, 128-byte swizzle: one copy moves a math warp's whole 32-row slab
+        const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), static_cast<uint64_t>(N / 64)};
+        const uint64_t str[2] = {static_cast<uint64_t>(N) * 2, 128};
+        const uint32_t box[3] = {64, 32, static_cast<uint32_t>(slab_blocks)};
+        if (!encode(&mp.d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, d, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return false;
+        if (c) {
+            if (!encode(&mp.c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, c, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+                return false;
+        } else {
+            mp.c = mp.d;   // never read when has_c == 0
+        }
+        return true;
     }
     {   // C, D: bf16 [G?][rows][N], box 64 x 32, 128-byte swizzle (one box row = 128 bytes)
         const uint64_t dims[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(rows), Gg};
@@ -293,7 +309,10 @@ dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *
     }
     p.num_tiles = (KIND == dg::KIND_MASKED || (KIND == dg::KIND_CONTIGUOUS && pair)) ? 0 : tiles;
     const int b_rows = pair ? bn / 2 : bn;
-    if (!build_maps(mp, a, sfa, b, c, d, rows, N, K, G, b_rows, batched)) return DG_ERR_INVALID_ARG;
+    // dense and contiguous D rows in whole 64-column blocks: one TMA copy per epilogue slab
+    p.cd_blocks = !batched && N % 64 == 0;
+    if (!build_maps(mp, a, sfa, b, c, d, rows, N, K, G, b_rows, batched, p.cd_blocks ? bn / 128 : 0))
+        return DG_ERR_INVALID_ARG;
     if (pair) {
         return launch_gemm<256, 4, KIND, true>(mp, p, tiles, di, st);
     }

@@ -64,6 +64,7 @@ struct GemmParams {
     int n_blocks;     // ceil(N/BN)
     int num_tiles;    // dense and unpaired contiguous tiles (others: derived on the device)
     int has_c;
+    int cd_blocks;    // 1: C and D maps are 3D {64 columns, rows, N/64 column blocks} (one copy per slab)
     const float *sfa;
     const float *sfb;
     const int32_t *grouped_layout;
@@ -449,12 +450,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 bulk_wait_group_read0();                         // the slab's last store has read it
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(&cfull[mw], L::SLAB_BYTES);
+                if (KIND != KIND_MASKED && p.cd_blocks) {
+                    tma_load_3d(&tm_c, &cfull[mw], slab, 0, srow0, col0 / 64);   // the whole slab
+                } else {
 #pragma unroll
-                for (int bx = 0; bx < HALF / 64; ++bx) {
-                    if (KIND == KIND_MASKED)
-                        tma_load_3d(&tm_c, &cfull[mw], slab + bx * 4096, col0 + bx * 64, srow0, ti.g);
-                    else
-                        tma_load_2d(&tm_c, &cfull[mw], slab + bx * 4096, col0 + bx * 64, srow0);
+                    for (int bx = 0; bx < HALF / 64; ++bx) {
+                        if (KIND == KIND_MASKED)
+                            tma_load_3d(&tm_c, &cfull[mw], slab + bx * 4096, col0 + bx * 64, srow0, ti.g);
+                        else
+                            tma_load_2d(&tm_c, &cfull[mw], slab + bx * 4096, col0 + bx * 64, srow0);
+                    }
                 }
             }
             float acc[HALF];
@@ -527,32 +532,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 __syncwarp();
             }
             // bf16 epilogue into the swizzled slab: row `lane`, 16-byte chunk ch of box bx lives
-            // at bx*4096 + lane*128 + ((ch ^ (lane & 7)) * 16).
+            // at bx*4096 + lane*128 + ((ch ^ (lane & 7)) * 16). A box's 8 C chunks are read before
+            // any is overwritten; C is added in packed fp32 pairs (a bf16 widens to fp32 exactly:
+            // low half << 16, high half with the low bits cleared).
 #pragma unroll
             for (int bx = 0; bx < HALF / 64; ++bx) {
+                uint4 cv[8];
+                if (do_c) {
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        cv[ch] = *reinterpret_cast<const uint4 *>(slab + bx * 4096 + lane * 128 + ((ch ^ (lane & 7)) * 16));
+                }
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    uint4 *pchunk = reinterpret_cast<uint4 *>(slab + bx * 4096 + lane * 128 + ((ch ^ (lane & 7)) * 16));
-                    float v[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = acc[bx * 64 + ch * 8 + e];
-                    if (do_c) {
-                        const uint4 cv = *pchunk;
-                        const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const __nv_bfloat162 c2 = *reinterpret_cast<const __nv_bfloat162 *>(&cw[e]);
-                            v[2 * e] += __bfloat162float(c2.x);
-                            v[2 * e + 1] += __bfloat162float(c2.y);
-                        }
-                    }
+                    const uint32_t cw[4] = {cv[ch].x, cv[ch].y, cv[ch].z, cv[ch].w};
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+                        float2 v = make_float2(acc[bx * 64 + ch * 8 + 2 * e], acc[bx * 64 + ch * 8 + 2 * e + 1]);
+                        if (do_c)
+                            v = __fadd2_rn(v, make_float2(__uint_as_float(cw[e] << 16), __uint_as_float(cw[e] & 0xFFFF0000u)));
+                        __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
                         w[e] = *reinterpret_cast<uint32_t *>(&h);
                     }
-                    *pchunk = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4 *>(slab + bx * 4096 + lane * 128 + ((ch ^ (lane & 7)) * 16)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
             if (KIND == KIND_MASKED) {
@@ -586,8 +590,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
+                    if (p.cd_blocks) {
+                        tma_store_3d(&tm_d, slab, 0, srow0, col0 / 64);   // the whole slab
+                    } else {
 #pragma unroll
-                    for (int bx = 0; bx < HALF / 64; ++bx) tma_store_2d(&tm_d, slab + bx * 4096, col0 + bx * 64, srow0);
+                        for (int bx = 0; bx < HALF / 64; ++bx) tma_store_2d(&tm_d, slab + bx * 4096, col0 + bx * 64, srow0);
+                    }
                     bulk_commit_group();
                 }
             }
