@@ -76,6 +76,32 @@ dg_status device_info(const DeviceInfo **out) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Launch configuration of every kernel: programmatic dependent launch (the kernel may start
+// while the previous kernel of the stream runs; it waits for it with griddepcontrol.wait before
+// touching global memory), plus a cluster shape when `cluster` > 1.
+struct Launch {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    Launch(dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster = 1) {
+        cfg.gridDim = grid;
+        cfg.blockDim = block;
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        int n = 1;
+        if (cluster > 1) {
+            attr[1].id = cudaLaunchAttributeClusterDimension;
+            attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
+            attr[1].val.clusterDim.y = 1;
+            attr[1].val.clusterDim.z = 1;
+            n = 2;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = n;
+    }
+};
+
 int pad4(int x) { return (x + 3) / 4 * 4; }
 
 uint64_t wait_limit_ns() {
@@ -228,19 +254,8 @@ dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p, int tiles, co
     static KernelInfo info[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    cfg.blockDim = dim3(dg::GEMM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = L::ALLOC;
-    cfg.stream = st;
-    if (PAIR) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
+    Launch ln(dim3(1, 1, 1), dim3(dg::GEMM_THREADS, 1, 1), L::ALLOC, st, PAIR ? 2 : 1);
+    cudaLaunchConfig_t &cfg = ln.cfg;
     KernelInfo &ki = info[dev];
     if (!ki.ready.load()) {
         std::lock_guard<std::mutex> lk(g_mu);
@@ -430,8 +445,8 @@ dg_status launch_swap(const SwapMaps &mp, const dg::SwapParams &p, long long til
     // them as its per-tile partial limit allows
     const long long grid = units < di->sm_count ? units : di->sm_count;
     if (grid <= 0) return DG_OK;
-    kern<<<static_cast<unsigned>(grid), L::THREADS, L::ALLOC, st>>>(mp.w, mp.x, mp.sfa, mp.c, p);
-    return from_cuda(cudaGetLastError());
+    Launch ln(dim3(static_cast<unsigned>(grid), 1, 1), dim3(L::THREADS, 1, 1), L::ALLOC, st);
+    return from_cuda(cudaLaunchKernelEx(&ln.cfg, kern, mp.w, mp.x, mp.sfa, mp.c, p));
 }
 
 // The few-row GEMM with the given stream-K scratch (partials for >= sm_count slots, flags zero).
@@ -565,9 +580,8 @@ dg_status dg_transform_sf(const float *sf_kmajor, float *sf_mnmajor, int batch, 
     const int ld = pad4(MN);
     if (ld == 0) return DG_OK;
     dim3 grid((ld + 31) / 32, (Kb + 31) / 32, batch);
-    dg::transform_sf_kernel<<<grid, dim3(32, 8), 0, static_cast<cudaStream_t>(stream)>>>(sf_kmajor, sf_mnmajor, MN,
-                                                                                         Kb, ld);
-    return from_cuda(cudaGetLastError());
+    Launch ln(grid, dim3(32, 8, 1), 0, static_cast<cudaStream_t>(stream));
+    return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::transform_sf_kernel, sf_kmajor, sf_mnmajor, MN, Kb, ld));
 }
 
 dg_status dg_cast_fp8_per_token(const void *x, void *q, float *sfa, int batch, int M, int K, void *stream) {
@@ -583,15 +597,18 @@ dg_status dg_cast_fp8_per_token(const void *x, void *q, float *sfa, int batch, i
     if (big_blocks >= 2LL * di->sm_count) {   // enough 32 x 4 blocks for two per SM
         dim3 grid((M + 31) / 32, (Kb + 3) / 4, batch);
         if (grid.y > 65535) return DG_ERR_INVALID_ARG;
-        dg::cast_per_token_kernel<32, 4><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x),
-                                                                 static_cast<uint8_t *>(q), sfa, M, K, pad4(M));
+        Launch ln(grid, dim3(256, 1, 1), 0, st);
+        return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_token_kernel<32, 4>,
+                                            static_cast<const __nv_bfloat16 *>(x), static_cast<uint8_t *>(q), sfa, M,
+                                            K, pad4(M)));
     } else {
         dim3 grid((M + 7) / 8, (Kb + 1) / 2, batch);
         if (grid.y > 65535) return DG_ERR_INVALID_ARG;
-        dg::cast_per_token_kernel<8, 2><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(x),
-                                                                static_cast<uint8_t *>(q), sfa, M, K, pad4(M));
+        Launch ln(grid, dim3(256, 1, 1), 0, st);
+        return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_token_kernel<8, 2>,
+                                            static_cast<const __nv_bfloat16 *>(x), static_cast<uint8_t *>(q), sfa, M,
+                                            K, pad4(M)));
     }
-    return from_cuda(cudaGetLastError());
 }
 
 dg_status dg_cast_fp8_per_block(const void *x, void *q, float *sfb, int batch, int N, int K, void *stream) {
@@ -603,9 +620,9 @@ dg_status dg_cast_fp8_per_block(const void *x, void *q, float *sfb, int batch, i
     if (s != DG_OK) return s;
     dim3 grid(K / 128, (N + 127) / 128, batch);
     if (grid.y > 65535) return DG_ERR_INVALID_ARG;
-    dg::cast_per_block_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const __nv_bfloat16 *>(x), static_cast<uint8_t *>(q), sfb, N, K);
-    return from_cuda(cudaGetLastError());
+    Launch ln(grid, dim3(256, 1, 1), 0, static_cast<cudaStream_t>(stream));
+    return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_block_kernel, static_cast<const __nv_bfloat16 *>(x),
+                                        static_cast<uint8_t *>(q), sfb, N, K));
 }
 
 int dg_sf_ld(int mn) { return mn <= 0 ? 0 : pad4(mn); }

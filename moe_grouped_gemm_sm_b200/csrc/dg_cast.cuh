@@ -14,6 +14,8 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include "dg_ptx.cuh"
+
 namespace dg {
 
 __device__ __forceinline__ uint4 ldg_stream_v4(const void *p) {
@@ -79,6 +81,8 @@ __global__ void __launch_bounds__(256) cast_per_token_kernel(const __nv_bfloat16
     const int Kb = K >> 7;
     const size_t bofs = static_cast<size_t>(blockIdx.z) * M;
     const int r0 = blockIdx.x * ROWS, kb0 = blockIdx.y * KBS;
+    pdl_launch_dependents();
+    pdl_wait();
 
     uint4 v[PER];
 #pragma unroll
@@ -126,6 +130,8 @@ __global__ void __launch_bounds__(256) cast_per_block_kernel(const __nv_bfloat16
     const size_t bofs = static_cast<size_t>(blockIdx.z) * N;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int chunk = t & 15, rbase = nb * 128 + (t >> 4);
+    pdl_launch_dependents();
+    pdl_wait();
 
     uint4 v[8];
 #pragma unroll
@@ -163,6 +169,8 @@ __global__ void __launch_bounds__(256) transform_sf_kernel(const float *__restri
     __shared__ float tile[32][33];
     const size_t b = blockIdx.z;
     const int m0 = blockIdx.x * 32, k0 = blockIdx.y * 32;
+    pdl_launch_dependents();
+    pdl_wait();
     for (int i = threadIdx.y; i < 32; i += 8) {
         const int m = m0 + i, k = k0 + threadIdx.x;
         tile[i][threadIdx.x] = (m < MN && k < Kb) ? in[(b * MN + m) * Kb + k] : 0.f;

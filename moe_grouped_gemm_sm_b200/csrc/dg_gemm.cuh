@@ -270,7 +270,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const bool leader = rank == 0;
     const int cid = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     const int ncid = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+    pdl_launch_dependents();
 
+    // prologue (overlaps the previous kernel's tail): barriers, descriptors, TMEM
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -297,10 +299,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tma_prefetch_desc(&tm_c);
         tma_prefetch_desc(&tm_d);
     }
-    if (PAIR_LIST && warp == 2) {
-        const int np = build_pair_list(p, pair_first, lane);
-        if (lane == 0) *num_pairs_smem = np;
-    }
     if (warp == 1) {
         if (PAIR) {
             tmem_alloc_pair(&ctx->tmem_base, L::TMEM_COLS);
@@ -309,6 +307,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tmem_alloc(&ctx->tmem_base, L::TMEM_COLS);
             tmem_relinquish();
         }
+    }
+    pdl_wait();   // from here on global memory may be read and written
+    if (PAIR_LIST && warp == 2) {
+        const int np = build_pair_list(p, pair_first, lane);
+        if (lane == 0) *num_pairs_smem = np;
     }
     tc_fence_before();
     if (PAIR)

@@ -173,10 +173,8 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    if (KIND == KIND_MASKED && blockIdx.x == 0 && threadIdx.x == 0) {
-        for (int gg = 0; gg < p.G; ++gg)
-            if (__ldg(p.masked_m + gg) > p.M) report_error(p.err, ERR_DATA);
-    }
+    pdl_launch_dependents();
+    // prologue (overlaps the previous kernel's tail): barriers, descriptors, TMEM
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -206,6 +204,11 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
     if (warp == 1) {
         tmem_alloc(&ctx->tmem_base, L::TMEM_COLS);
         tmem_relinquish();
+    }
+    pdl_wait();   // from here on global memory may be read and written
+    if (KIND == KIND_MASKED && blockIdx.x == 0 && threadIdx.x == 0) {
+        for (int gg = 0; gg < p.G; ++gg)
+            if (__ldg(p.masked_m + gg) > p.M) report_error(p.err, ERR_DATA);
     }
     tc_fence_before();
     __syncthreads();

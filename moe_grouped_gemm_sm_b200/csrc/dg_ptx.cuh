@@ -25,6 +25,18 @@ __device__ __forceinline__ void report_error(int *err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
 
+// Programmatic dependent launch: every kernel of the library is launched so that it may start
+// while the previous kernel of its stream is still running. launch_dependents lets the next
+// kernel start early; wait blocks until the previous kernel has finished and its memory is
+// visible, and is executed by every thread before its first global memory access (the
+// library cannot know what the previous kernel wrote). Without such a dependency both are
+// no-ops.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Flags between CTAs of one grid (global memory, gpu scope): a release store publishes the
 // writer's earlier stores (made visible gpu-wide by a fence), an acquire load sees them.
 __device__ __forceinline__ void flag_store_release(int *p, int v) {
