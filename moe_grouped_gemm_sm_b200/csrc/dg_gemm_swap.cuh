@@ -25,8 +25,8 @@
 //
 // CTA layout: warps 0, 2, 3 TMA producers (weights and activations on two threads each, the A
 // scales on four), warp 1 TMEM allocator + single-thread tcgen05.mma issuer (kind::f8f6f4,
-// M = 128, N = TN), warps 4.. TN/64 math warpgroups (thread = weight row, registers = its
-// warpgroup's 64 token columns).
+// M = 128, N = TN), warps 4-11 two math warpgroups (thread = weight row, registers = its
+// warpgroup's TN/2 token columns).
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -57,14 +57,14 @@ struct SwapParams {
 template <int TN, int STAGES>
 struct SwapLayout {
     static_assert(TN == 64 || TN == 128, "token tile");
-    static constexpr int NWG = TN / 64;                      // math warpgroups, 64 token columns each
-    static constexpr int COLS = TN / NWG;                    // token columns per math warpgroup
+    static constexpr int NWG = 2;                            // math warpgroups: two warps per SM sub-partition
+    static constexpr int COLS = TN / NWG;                    // token columns per math warpgroup (32 or 64)
     static constexpr int THREADS = 128 + 128 * NWG;
     static constexpr int W_BYTES = 128 * BK;                 // weight tile: 128 rows x 128 B
     static constexpr int X_BYTES = TN * BK;                  // activation tile: TN rows x 128 B
     static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
     static constexpr int NBUF = (512 / TN) > 4 ? 4 : (512 / TN);
-    static constexpr int SFS = STAGES + NBUF + 1;            // A-scale ring, own full/empty barriers
+    static constexpr int SFS = 16;                           // A-scale ring (a power of two), own barriers
     static constexpr int OFF_W = 0;
     static constexpr int OFF_X = OFF_W + STAGES * W_BYTES;
     static constexpr int OFF_SFA = OFF_X + STAGES * X_BYTES;
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
         // ---------------- math warpgroups: promotion, partials, tile epilogue ----------------
         // Every math thread walks the same segments and meets the same named barriers, even
         // after a wait has given up (then the work is skipped), so no barrier is left waiting.
-        const int wg = (warp - 4) >> 2;                    // token columns [wg·64, wg·64 + 64)
+        const int wg = (warp - 4) >> 2;                    // token columns [wg·COLS, wg·COLS + COLS)
         const int q = warp & 3;                            // TMEM lane quadrant = weight rows 32q..
         const int n = q * 32 + lane;                       // this thread's weight row in the tile
         const int c_self = static_cast<int>(blockIdx.x);

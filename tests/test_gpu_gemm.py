@@ -45,6 +45,17 @@ def test_dense_small_full_compare(oracle, M, N, K, with_c):
     assert_close(bf16_host_f64(d), ref, f"{M}x{N}x{K} c={with_c}")
 
 
+@pytest.mark.parametrize("M,N,K", [(512, 10240, 256), (400, 10176, 384)])
+def test_dense_partial_last_wave(oracle, M, N, K):
+    """More 256 x 256 pair tiles than one wave of resident CTA pairs, the last wave partial,
+    with ragged rows and columns."""
+    dv, hv = quantised(oracle, M, N, K, True, salt=M + N)
+    a, sfa, b, sfb, c = dv
+    d = ops.fp8_gemm_nt(a, sfa, b, sfb, c)
+    torch.cuda.synchronize()
+    assert_close(bf16_host_f64(d), oracle.gemm_nt(*hv), f"{M}x{N}x{K} last wave")
+
+
 def test_dense_c_aliases_d(oracle):
     M, N, K = 192, 384, 512
     dv, hv = quantised(oracle, M, N, K, True, salt=9)
