@@ -322,53 +322,104 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
             const float *sfb_col = p.sfb + (static_cast<size_t>(g) * p.Nb + nt) * p.Kb;
             float sb_win = kbs + lane < kbe ? __ldg(sfb_col + kbs + lane) : 0.f;
             float sb_nxt = kbs + 32 + lane < kbe ? __ldg(sfb_col + kbs + 32 + lane) : 0.f;
-            for (int i = 0; i < kbe - kbs; ++i, ++it) {
-                const int b = it % NBUF;
-                const int j = it % L::SFS;
+            const int nk = kbe - kbs;
+            // fold one K block's partial (in registers rr) into acc: acc += P · sfa[col] · sb
+            auto fold = [&](const uint32_t (&rr)[32], int c, const float *sfa_row, float sb) {
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    // four token columns: their A scales (broadcast from shared memory) times sb
+                    const float4 sa4 = *reinterpret_cast<const float4 *>(sfa_row + c * 32 + v * 4);
+                    const float2 s01 = __fmul2_rn(make_float2(sa4.x, sa4.y), make_float2(sb, sb));
+                    const float2 s23 = __fmul2_rn(make_float2(sa4.z, sa4.w), make_float2(sb, sb));
+                    const int e = c * 32 + v * 4;
+                    const float2 a01 = __ffma2_rn(make_float2(__uint_as_float(rr[v * 4]), __uint_as_float(rr[v * 4 + 1])),
+                                                  s01, make_float2(acc[e], acc[e + 1]));
+                    const float2 a23 = __ffma2_rn(make_float2(__uint_as_float(rr[v * 4 + 2]), __uint_as_float(rr[v * 4 + 3])),
+                                                  s23, make_float2(acc[e + 2], acc[e + 3]));
+                    acc[e] = a01.x;
+                    acc[e + 1] = a01.y;
+                    acc[e + 2] = a23.x;
+                    acc[e + 3] = a23.y;
+                }
+            };
+            auto sb_of = [&](int i) {                      // sfb of K block kbs + i (all lanes)
                 if ((i & 31) == 0 && i > 0) {
                     sb_win = sb_nxt;
                     sb_nxt = kbs + i + 32 + lane < kbe ? __ldg(sfb_col + kbs + i + 32 + lane) : 0.f;
                 }
-                const float sb = __shfl_sync(0xFFFFFFFFu, sb_win, i & 31);
-                if (!ok) continue;
-                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], (it / NBUF) & 1, ctx));
-                if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sfa_full[j], (it / L::SFS) & 1, ctx));
-                if (!ok) continue;
-                tc_fence_after();
-                const float *sfa_row = sfa_ring + j * TN + wg * COLS;
-                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                       static_cast<uint32_t>(b * TN + wg * COLS);
-                uint32_t r[2][32];
-                tmem_ld32(taddr, r[0]);
-                tmem_ld_wait_regs32(r[0]);
-#pragma unroll
-                for (int c = 0; c < COLS / 32; ++c) {
-                    if (c + 1 < COLS / 32) tmem_ld32(taddr + (c + 1) * 32, r[(c + 1) & 1]);
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        // four token columns: their A scales (broadcast from shared memory) times sb
-                        const float4 sa4 = *reinterpret_cast<const float4 *>(sfa_row + c * 32 + v * 4);
-                        const float2 s01 = __fmul2_rn(make_float2(sa4.x, sa4.y), make_float2(sb, sb));
-                        const float2 s23 = __fmul2_rn(make_float2(sa4.z, sa4.w), make_float2(sb, sb));
-                        const int e = c * 32 + v * 4;
-                        const float2 a01 = __ffma2_rn(make_float2(__uint_as_float(r[c & 1][v * 4]),
-                                                                  __uint_as_float(r[c & 1][v * 4 + 1])),
-                                                      s01, make_float2(acc[e], acc[e + 1]));
-                        const float2 a23 = __ffma2_rn(make_float2(__uint_as_float(r[c & 1][v * 4 + 2]),
-                                                                  __uint_as_float(r[c & 1][v * 4 + 3])),
-                                                      s23, make_float2(acc[e + 2], acc[e + 3]));
-                        acc[e] = a01.x;
-                        acc[e + 1] = a01.y;
-                        acc[e + 2] = a23.x;
-                        acc[e + 3] = a23.y;
-                    }
-                    if (c + 1 < COLS / 32) tmem_ld_wait_regs32(r[(c + 1) & 1]);
-                }
+                return __shfl_sync(0xFFFFFFFFu, sb_win, i & 31);
+            };
+            auto ready = [&](uint32_t itx) {               // TMEM buffer and A scales of itx (warp-uniform)
+                bool r = __all_sync(0xFFFFFFFFu, mbar_wait(&tfull[itx % NBUF], (itx / NBUF) & 1, ctx));
+                if (r) r = __all_sync(0xFFFFFFFFu, mbar_wait(&sfa_full[itx % L::SFS], (itx / L::SFS) & 1, ctx));
+                return r;
+            };
+            auto taddr_of = [&](uint32_t itx) {
+                return tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                       static_cast<uint32_t>((itx % NBUF) * TN + wg * COLS);
+            };
+            auto release = [&](uint32_t itx) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive_relaxed(&sfa_empty[j]);
-                    mbar_arrive_relaxed(&tempty[b]);
+                    mbar_arrive_relaxed(&sfa_empty[itx % L::SFS]);
+                    mbar_arrive_relaxed(&tempty[itx % NBUF]);
+                }
+            };
+            if constexpr (COLS == 32) {
+                // one 32-column TMEM load per K block, software-pipelined across K blocks: the
+                // next block's load is in flight while the current block is folded in
+                uint32_t r0[32], r1[32];
+                auto step = [&](uint32_t (&cur)[32], uint32_t (&nxt)[32], int i) {
+                    const float sb = sb_of(i);
+                    if (!ok) return;
+                    tmem_ld_wait_regs32(cur);              // block i is in registers
+                    const uint32_t itn = it + 1;
+                    if (i + 1 < nk) {
+                        ok = ready(itn);
+                        if (ok) {
+                            tc_fence_after();
+                            tmem_ld32(taddr_of(itn), nxt);
+                        }
+                    }
+                    fold(cur, 0, sfa_ring + (it % L::SFS) * TN + wg * COLS, sb);
+                    release(it);
+                };
+                if (ok && nk > 0) {
+                    ok = ready(it);
+                    if (ok) {
+                        tc_fence_after();
+                        tmem_ld32(taddr_of(it), r0);
+                    }
+                }
+                for (int i = 0; i < nk; i += 2) {
+                    step(r0, r1, i);
+                    ++it;
+                    if (i + 1 < nk) {
+                        step(r1, r0, i + 1);
+                        ++it;
+                    }
+                }
+                if (ok) tmem_ld_wait_regs32(r0);           // nothing is left in flight
+            } else {
+                for (int i = 0; i < nk; ++i, ++it) {
+                    const float sb = sb_of(i);
+                    if (!ok) continue;
+                    ok = ready(it);
+                    if (!ok) continue;
+                    tc_fence_after();
+                    const float *sfa_row = sfa_ring + (it % L::SFS) * TN + wg * COLS;
+                    const uint32_t taddr = taddr_of(it);
+                    uint32_t r[2][32];
+                    tmem_ld32(taddr, r[0]);
+                    tmem_ld_wait_regs32(r[0]);
+#pragma unroll
+                    for (int c = 0; c < COLS / 32; ++c) {
+                        if (c + 1 < COLS / 32) tmem_ld32(taddr + (c + 1) * 32, r[(c + 1) & 1]);
+                        fold(r[c & 1], c, sfa_row, sb);
+                        if (c + 1 < COLS / 32) tmem_ld_wait_regs32(r[(c + 1) & 1]);
+                    }
+                    release(it);
                 }
             }
             if (!owner) {
