@@ -155,6 +155,19 @@ int forced_swap() {
     return v;
 }
 
+// Failure test only (DG_TEST_SKIP_RELEASE=1): the tile GEMM withholds one TMEM-buffer release,
+// so that a pipeline wait runs out of time and reports DG_ERR_TIMEOUT without faulting.
+int test_skip_release() {
+    static std::atomic<int> cached{-1};
+    int v = cached.load();
+    if (v < 0) {
+        const char *s = std::getenv("DG_TEST_SKIP_RELEASE");
+        v = s && std::atoi(s) ? 1 : 0;
+        cached.store(v);
+    }
+    return v;
+}
+
 // Encodes a tiled tensor map. dims/box are innermost first; strides (bytes) for dims 1..rank-1.
 bool encode(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
             const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle sw) {
@@ -304,6 +317,7 @@ dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.err = di->err;
     p.timeout_ns = wait_limit_ns();
+    p.test_skip_release = test_skip_release();
     const bool batched = KIND == dg::KIND_MASKED;
     const int fbn = forced_bn();
     const int bn = fbn ? fbn : (N > 128 ? 256 : 128);

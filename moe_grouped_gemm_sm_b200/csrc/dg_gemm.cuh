@@ -65,6 +65,7 @@ struct GemmParams {
     int num_tiles;    // dense and unpaired contiguous tiles (others: derived on the device)
     int has_c;
     int cd_blocks;    // 1: C and D maps are 3D {64 columns, rows, N/64 column blocks} (one copy per slab)
+    int test_skip_release;   // failure test only: warp 4 of CTA 0 skips its first TMEM release
     const float *sfa;
     const float *sfb;
     const int32_t *grouped_layout;
@@ -516,8 +517,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                // TMEM reads are complete (wait::ld) and sa was consumed: a relaxed arrive suffices
-                if (lane == 0) {
+                // TMEM reads are complete (wait::ld) and sa was consumed: a relaxed arrive suffices.
+                // (A failure test can withhold one release: the MMA's bounded wait then runs out.)
+                if (lane == 0 && !(p.test_skip_release && blockIdx.x == 0 && warp == 4 && it == 0)) {
                     if (PAIR)
                         mbar_arrive_cluster_relaxed(tempty_leader0 + b * 8);
                     else

@@ -1,0 +1,107 @@
+"""Failure detection without a GPU fault: bad data that only the device can see, and a pipeline
+wait that runs out of time. Each sets the per-device error word, which dg_get_device_error()
+returns (and clears); the work that is still well-defined is done, and the context stays usable.
+"""
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+from moe_grouped_gemm_sm_b200 import _lib, build, ops, synth
+from tests.gpu_util import assert_close, bf16_dev, bf16_host_f64, dev, host
+
+pytestmark = pytest.mark.gpu
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CHILD = os.environ.get("DG_TEST_SKIP_RELEASE") == "1"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+@pytest.mark.skipif(CHILD, reason="parent-process test")
+def test_contiguous_expert_id_out_of_range(oracle):
+    """A 128-row block whose expert id is >= G: the error word says DG_ERR_DEVICE, that block is
+    skipped, and every other block is computed as usual."""
+    G, N, K = 4, 264, 256
+    m, layout, x, w = synth.contiguous_inputs(G, N, K, lo=200, hi=300, salt=31)
+    layout = layout.copy()
+    bad = 2 * 128                                         # third 128-row block
+    assert layout[bad] >= 0
+    layout[bad:bad + 128] = G + 1
+    a, sfa = ops.cast_per_token(bf16_dev(x))
+    b, sfb = ops.cast_per_block(bf16_dev(w))
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+    d = ops.m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, dev(layout))
+    torch.cuda.synchronize()
+    assert _lib.dg_get_device_error() == _lib.DG_ERR_DEVICE
+    assert _lib.dg_get_device_error() == _lib.DG_OK       # read and cleared
+    ok_layout = layout.copy()
+    ok_layout[bad:bad + 128] = -1                         # the oracle's view: no expert there
+    rows = np.nonzero(ok_layout >= 0)[0].astype(np.int32)
+    ref = oracle.m_grouped_contiguous(host(a), host(sfa), host(b), host(sfb), ok_layout, None, rows=rows)
+    assert_close(bf16_host_f64(d)[rows], ref, "contiguous with one bad block")
+
+
+@pytest.mark.skipif(CHILD, reason="parent-process test")
+def test_masked_m_above_m_max(oracle):
+    """masked_m[g] > M_max: the error word says DG_ERR_DEVICE and the expert is computed as if
+    masked_m[g] were M_max."""
+    G, M_max, N, K = 3, 160, 264, 256
+    masked_m, a_bits, w = synth.masked_inputs(G, M_max, N, K, lo=10, hi=160, salt=32)
+    a, sfa = ops.cast_per_token(bf16_dev(a_bits))
+    b, sfb = ops.cast_per_block(bf16_dev(w))
+    given = masked_m.copy()
+    given[1] = M_max + 5
+    d = bf16_dev(np.full((G, M_max, N), synth.sentinel_bf16(), np.uint16))
+    ops.m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, dev(given), 192, out=d)
+    torch.cuda.synchronize()
+    assert _lib.dg_get_device_error() == _lib.DG_ERR_DEVICE
+    clamped = given.copy()
+    clamped[1] = M_max
+    ref = oracle.m_grouped_masked(host(a), host(sfa), host(b), host(sfb), clamped)
+    dh = bf16_host_f64(d)
+    for g in range(G):
+        assert_close(dh[g, :clamped[g]], ref[g, :clamped[g]], f"masked expert {g}")
+
+
+@pytest.mark.skipif(CHILD, reason="parent-process test")
+def test_pipeline_wait_timeout_is_reported():
+    """A child process withholds one TMEM-buffer release in the tile GEMM (a debug-only switch)
+    with a 100 ms wait limit: the MMA issuer's wait runs out, the kernel stops and returns, and
+    DG_ERR_TIMEOUT is reported; the context then still computes correctly."""
+    env = dict(os.environ, DG_TEST_SKIP_RELEASE="1", DG_WAIT_TIMEOUT_MS="100")
+    cmd = [sys.executable, "-m", "pytest", os.path.join(HERE, "test_gpu_failure.py"), "-q", "-x", "-m", "gpu",
+           "-k", "child"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    tail = "\n".join((r.stdout + r.stderr).splitlines()[-25:])
+    assert r.returncode == 0 and " passed" in r.stdout, tail
+
+
+@pytest.mark.skipif(not CHILD, reason="runs in the child process of test_pipeline_wait_timeout_is_reported")
+def test_child_timeout_then_recovery(oracle):
+    M, N, K = 512, 512, 1024                              # CTA-pair tiles, several K blocks
+    x, w, c = synth.dense_inputs(M, N, K, False, salt=41)
+    a, sfa = ops.cast_per_token(bf16_dev(x))
+    b, sfb = ops.cast_per_block(bf16_dev(w))
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+    ops.fp8_gemm_nt(a, sfa, b, sfb, None)
+    torch.cuda.synchronize()
+    assert _lib.dg_get_device_error() == _lib.DG_ERR_TIMEOUT
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+    # the context is usable: a few-row GEMM (another kernel, no withheld release) is exact
+    M2, N2, K2 = 64, 2112, 7168
+    x2, w2, _ = synth.dense_inputs(M2, N2, K2, False, salt=42)
+    a2, sfa2 = ops.cast_per_token(bf16_dev(x2))
+    b2, sfb2 = ops.cast_per_block(bf16_dev(w2))
+    d2 = ops.fp8_gemm_nt(a2, sfa2, b2, sfb2, None)
+    torch.cuda.synchronize()
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+    ref = oracle.gemm_nt(host(a2), host(sfa2), host(b2), host(sfb2), None)
+    assert_close(bf16_host_f64(d2), ref, "after a timeout")
