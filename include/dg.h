@@ -66,19 +66,22 @@ typedef enum dg_status {
  *   b   e4m3 [N,K] row-major;          sfb fp32 [Nb][Kb]
  *   c   bf16 [M,N] row-major or NULL (then C = 0); may alias d
  *   d   bf16 [M,N] row-major, written in full.
- * M may be 0 (nothing is queued). For M <= 128 the work is split over every SM and the
- * partial sums meet in a library-owned workspace of the (device, stream) pair, allocated
- * (cudaMalloc, sm_count x 64 KB) by the pair's first such call and kept until the process
- * ends; a first call made under CUDA-graph capture cannot allocate and computes with the
- * tile kernel instead (same result within the stated bound). */
+ * M may be 0 (nothing is queued). For M <= 128 the K blocks are split over several SMs:
+ *   - with few 128-column tiles (at most 64) and K <= 8192, over a thread-block cluster per
+ *     tile, whose partial sums meet in distributed shared memory (no scratch at all);
+ *   - otherwise over every SM (stream-K), whose partial sums meet in a library-owned
+ *     workspace of the (device, stream) pair, allocated (cudaMalloc, sm_count x 64 KB) by
+ *     the pair's first such call and kept until the process ends; a first call made under
+ *     CUDA-graph capture cannot allocate and computes with the tile kernel instead.
+ * Every choice gives the same result within the stated bound, and each is deterministic. */
 DG_API dg_status dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const float *sfb,
                          const void *c, void *d, int M, int N, int K, void *stream);
 
-/* dg_fp8_gemm_nt for M <= 128 without any allocation. Same arguments, and the same result bit
- * for bit (the same kernel and the same split of the work), but the kernel's scratch (the
- * partial sums and their flags) is a fixed static device array of the library instead of a
- * per-stream workspace, so the call never allocates and may be made under graph capture on
- * any stream. That array is shared by all streams of a device: calls of this entry point must
+/* dg_fp8_gemm_nt's stream-K path for M <= 128 without any allocation. Same arguments, and the
+ * same result bit for bit as dg_fp8_gemm_nt whenever that call takes the stream-K kernel (the
+ * same kernel and the same split of the work), but the kernel's scratch (the partial sums and
+ * their flags) is a fixed static device array of the library instead of a per-stream
+ * workspace, so the call never allocates and may be made under graph capture on any stream. That array is shared by all streams of a device: calls of this entry point must
  * not run concurrently on one device. The pages have no counterpart of this entry point.
  * Errors: those of dg_fp8_gemm_nt, plus DG_ERR_UNSUPPORTED (nothing queued) when M > 128 or
  * when the device has more than 256 SMs (the array's capacity). */

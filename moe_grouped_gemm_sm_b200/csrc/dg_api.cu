@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstdlib>
@@ -14,6 +15,7 @@
 #include "../../include/dg.h"
 #include "dg_cast.cuh"
 #include "dg_gemm.cuh"
+#include "dg_gemm_splitk.cuh"
 #include "dg_gemm_swap.cuh"
 
 namespace {
@@ -82,7 +84,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct Launch {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
-    Launch(dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster = 1) {
+    Launch(dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster = 1, bool cluster_attr = false) {
         cfg.gridDim = grid;
         cfg.blockDim = block;
         cfg.dynamicSmemBytes = smem;
@@ -90,7 +92,7 @@ struct Launch {
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         int n = 1;
-        if (cluster > 1) {
+        if (cluster > 1 || cluster_attr) {
             attr[1].id = cudaLaunchAttributeClusterDimension;
             attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
             attr[1].val.clusterDim.y = 1;
@@ -153,6 +155,37 @@ int forced_swap() {
         cached.store(v);
     }
     return v;
+}
+
+// Cluster size of the few-row split-K kernel for tests and experiments (DG_SPLITK_S=1|2|3|4|6|8|16);
+// 0 = cost model. A forced size that the shape or the device cannot take falls back to the model.
+int forced_splitk_s() {
+    static std::atomic<int> cached{-1};
+    int v = cached.load();
+    if (v < 0) {
+        v = 0;
+        if (const char *s = std::getenv("DG_SPLITK_S")) v = std::atoi(s);
+        if (v != 1 && v != 2 && v != 3 && v != 4 && v != 6 && v != 8 && v != 16) v = 0;
+        cached.store(v);
+    }
+    return v;
+}
+
+// Few-row kernel by shape: the cluster split-K kernel when every tile fits one round of
+// clusters with a moderate K (its partials never leave the chip), stream-K otherwise (it splits
+// any tile count evenly over every SM, at the cost of a reduction through global memory).
+// DG_FEW_ROW=streamk|cluster overrides.
+bool use_streamk(int groups, int m_tiles, int N, int K) {
+    static std::atomic<int> cached{-1};
+    int v = cached.load();
+    if (v < 0) {
+        const char *s = std::getenv("DG_FEW_ROW");
+        v = s && std::strcmp(s, "streamk") == 0 ? 1 : (s && std::strcmp(s, "cluster") == 0 ? 2 : 0);
+        cached.store(v);
+    }
+    if (v) return v == 1;
+    const long long tiles = static_cast<long long>(groups) * m_tiles * ((N + 127) / 128);
+    return tiles > 64 || K / 128 > 64;
 }
 
 // Failure test only (DG_TEST_SKIP_RELEASE=1): the tile GEMM withholds one TMEM-buffer release,
@@ -513,6 +546,106 @@ dg_status run_swap(const void *a, const float *sfa, const void *b, const float *
     return run_swap_with<KIND>(a, sfa, b, sfb, c, d, masked_m, expected_m, rows, N, K, G, st, di, w.ws, w.flags);
 }
 
+// ---- few-row GEMMs: cluster split-K (dg_gemm_splitk.cuh) ----
+// Per (kernel, device): how many clusters of each size S = 1, 2, 4, 8, 16 can be resident.
+constexpr int kSplitSizes[7] = {1, 2, 3, 4, 6, 8, 16};   // cluster sizes the kernel takes
+struct SplitInfo {
+    std::atomic<int> ready{0};
+    int max_clusters[7] = {0, 0, 0, 0, 0, 0, 0};
+};
+
+template <int TN, int STAGES, int KIND>
+dg_status launch_splitk(const SwapMaps &mp, const dg::SwapParams &p, int tiles, const DeviceInfo *di,
+                        cudaStream_t st) {
+    using L = dg::SplitLayout<TN, STAGES>;
+    auto kern = dg::gemm_splitk_kernel<TN, STAGES, KIND>;
+    static SplitInfo info[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
+    SplitInfo &si = info[dev];
+    if (!si.ready.load()) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!si.ready.load()) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC) != cudaSuccess)
+                return DG_ERR_CUDA;
+            const bool big = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+            si.max_clusters[0] = di->sm_count;
+            for (int i = 1; i < 7; ++i) {
+                const int S = kSplitSizes[i];
+                if (S > 8 && !big) break;
+                Launch ln(dim3(static_cast<unsigned>(S * (di->sm_count / S)), 1, 1), dim3(L::THREADS, 1, 1), L::ALLOC, st, S);
+                int n = 0;
+                if (cudaOccupancyMaxActiveClusters(&n, kern, &ln.cfg) != cudaSuccess) {
+                    cudaGetLastError();
+                    n = 0;
+                }
+                si.max_clusters[i] = n;
+            }
+            si.ready.store(1);
+        }
+    }
+    // Cluster size: the modelled time (cycles) of the busiest CTA, rounds x (its K blocks at the
+    // rate one SM streams from HBM, ~26 B/clk with this ring depth, which is also every SM's
+    // share of the full HBM rate) plus one reduction tail per round.
+    const double kb_bytes = 128.0 * 128 + TN * 128;
+    int best_s = 0, best_c = 0;
+    double best_t = 0;
+    for (int i = 0; i < 7; ++i) {
+        const int S = kSplitSizes[i];
+        if (S > p.Kb || si.max_clusters[i] <= 0) continue;
+        const int C = si.max_clusters[i] < tiles ? si.max_clusters[i] : tiles;
+        const int rounds = (tiles + C - 1) / C;
+        const double per_cta = static_cast<double>(rounds) * ((p.Kb + S - 1) / S);
+        const double t = per_cta * kb_bytes / 26.0 + (S > 1 ? 3000.0 : 1500.0) * rounds;
+        if (best_s == 0 || t < best_t || S == forced_splitk_s()) {
+            best_s = S;
+            best_c = C;
+            best_t = t;
+            if (S == forced_splitk_s()) break;
+        }
+    }
+    if (best_s == 0) return DG_ERR_UNSUPPORTED;
+    Launch ln(dim3(static_cast<unsigned>(best_c * best_s), 1, 1), dim3(L::THREADS, 1, 1), L::ALLOC, st, best_s, true);
+    return from_cuda(cudaLaunchKernelEx(&ln.cfg, kern, mp.w, mp.x, mp.sfa, p));
+}
+
+template <int KIND>
+dg_status run_splitk(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
+                     const int32_t *masked_m, int expected_m, int rows, int N, int K, int G, cudaStream_t st) {
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    const bool batched = KIND == dg::KIND_MASKED;
+    const int hint = batched ? (expected_m > 0 ? expected_m : rows) : rows;
+    const int tn = hint <= 64 ? 64 : 128;
+    dg::SwapParams p{};
+    p.M = rows;
+    p.N = N;
+    p.K = K;
+    p.G = G;
+    p.Kb = K / 128;
+    p.Nb = (N + 127) / 128;
+    p.ld_sfa = pad4(rows);
+    p.n_tiles = (N + 127) / 128;
+    p.m_tiles = (rows + tn - 1) / tn;
+    p.has_c = c != nullptr;
+    p.sfb = sfb;
+    p.masked_m = masked_m;
+    p.c = static_cast<const __nv_bfloat16 *>(c);
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.err = di->err;
+    p.timeout_ns = wait_limit_ns();
+    // tiles the cluster count is sized for: the masked layout's real count depends on masked_m,
+    // estimated from expected_m
+    const int m_est = batched ? (hint + tn - 1) / tn : p.m_tiles;
+    const long long tiles = static_cast<long long>(batched ? G : 1) * (m_est < 1 ? 1 : m_est) * p.n_tiles;
+    if (tiles > (1 << 30)) return DG_ERR_INVALID_ARG;
+    SwapMaps mp;
+    if (!build_swap_maps(mp, a, sfa, b, nullptr, rows, N, K, G, tn, batched)) return DG_ERR_INVALID_ARG;
+    if (tn == 64) return launch_splitk<64, 7, KIND>(mp, p, static_cast<int>(tiles), di, st);
+    return launch_splitk<128, 4, KIND>(mp, p, static_cast<int>(tiles), di, st);
+}
+
 dg_status check_gemm_common(const void *a, const float *sfa, const void *b, const float *sfb, const void *c,
                             const void *d, int N, int K) {
     if (!a || !sfa || !b || !sfb || !d) return DG_ERR_INVALID_ARG;
@@ -535,8 +668,11 @@ dg_status dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const f
     if (M == 0) return DG_OK;
     const int fs = forced_swap();
     if (fs >= 0 ? fs == 1 && M <= 128 : M <= 128) {
-        const dg_status r = run_swap<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, 0, M, N, K, 1,
-                                                     static_cast<cudaStream_t>(stream));
+        const dg_status r = use_streamk(1, 1, N, K)
+                                ? run_swap<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, 0, M, N, K, 1,
+                                                           static_cast<cudaStream_t>(stream))
+                                : run_splitk<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, 0, M, N, K, 1,
+                                                             static_cast<cudaStream_t>(stream));
         if (r != DG_ERR_UNSUPPORTED) return r;
     }
     return run_gemm<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, nullptr, M, N, K, 1,
@@ -577,8 +713,11 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const
     if (s != DG_OK) return s;
     if (M_max == 0) return DG_OK;
     if (forced_swap() == 1) {   // the pair kernel streams the masked page shapes faster
-        const dg_status r = run_swap<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, masked_m, expected_m, M_max, N, K, G,
-                                                      static_cast<cudaStream_t>(stream));
+        const dg_status r = use_streamk(G, 1, N, K)
+                                ? run_swap<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, masked_m, expected_m, M_max, N, K,
+                                                            G, static_cast<cudaStream_t>(stream))
+                                : run_splitk<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, masked_m, expected_m, M_max, N,
+                                                              K, G, static_cast<cudaStream_t>(stream));
         if (r != DG_ERR_UNSUPPORTED) return r;
     }
     return run_gemm<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, nullptr, masked_m, M_max, N, K, G,

@@ -225,17 +225,33 @@ __device__ __forceinline__ int build_pair_list(const GemmParams &p, uint16_t *pa
     return count;
 }
 
-// tcgen05.wait::ld with the loaded registers as in/out operands, so that no use of them can
-// be scheduled before the wait.
+// tcgen05.wait::ld, then the loaded registers are read. The reads sit in the same asm statement
+// as the wait, with separate input and output operands: tied in/out operands would allow the
+// compiler to copy a register that the asynchronous load has not written yet in front of the
+// wait, and a bare wait would allow it to move uses above the wait.
 __device__ __forceinline__ void tmem_ld_wait_regs32(uint32_t (&r)[32]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
-                   "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
-                   "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-                 :
-                 : "memory");
+    uint32_t t[32];
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;\n\t"
+        "mov.b32 %0, %32;\n\tmov.b32 %1, %33;\n\tmov.b32 %2, %34;\n\tmov.b32 %3, %35;\n\t"
+        "mov.b32 %4, %36;\n\tmov.b32 %5, %37;\n\tmov.b32 %6, %38;\n\tmov.b32 %7, %39;\n\t"
+        "mov.b32 %8, %40;\n\tmov.b32 %9, %41;\n\tmov.b32 %10, %42;\n\tmov.b32 %11, %43;\n\t"
+        "mov.b32 %12, %44;\n\tmov.b32 %13, %45;\n\tmov.b32 %14, %46;\n\tmov.b32 %15, %47;\n\t"
+        "mov.b32 %16, %48;\n\tmov.b32 %17, %49;\n\tmov.b32 %18, %50;\n\tmov.b32 %19, %51;\n\t"
+        "mov.b32 %20, %52;\n\tmov.b32 %21, %53;\n\tmov.b32 %22, %54;\n\tmov.b32 %23, %55;\n\t"
+        "mov.b32 %24, %56;\n\tmov.b32 %25, %57;\n\tmov.b32 %26, %58;\n\tmov.b32 %27, %59;\n\t"
+        "mov.b32 %28, %60;\n\tmov.b32 %29, %61;\n\tmov.b32 %30, %62;\n\tmov.b32 %31, %63;"
+        : "=r"(t[0]), "=r"(t[1]), "=r"(t[2]), "=r"(t[3]), "=r"(t[4]), "=r"(t[5]), "=r"(t[6]), "=r"(t[7]),
+          "=r"(t[8]), "=r"(t[9]), "=r"(t[10]), "=r"(t[11]), "=r"(t[12]), "=r"(t[13]), "=r"(t[14]), "=r"(t[15]),
+          "=r"(t[16]), "=r"(t[17]), "=r"(t[18]), "=r"(t[19]), "=r"(t[20]), "=r"(t[21]), "=r"(t[22]), "=r"(t[23]),
+          "=r"(t[24]), "=r"(t[25]), "=r"(t[26]), "=r"(t[27]), "=r"(t[28]), "=r"(t[29]), "=r"(t[30]), "=r"(t[31])
+        : "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = t[i];
 }
 
 template <int BN, int STAGES, int KIND, bool PAIR>
@@ -491,8 +507,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 const float sa = sfa_ring[j * BM + q * 32 + lane];
                 tc_fence_after();
                 const float scale = sa * sb;
+                // the slot is read: the generic-proxy read is ordered before the producer's next
+                // TMA write into the slot (async proxy) by a proxy fence, which release/acquire
+                // through the mbarrier alone does not give
+                fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_relaxed(&sfa_empty[j]);   // the slot is read
+                if (lane == 0) mbar_arrive_relaxed(&sfa_empty[j]);
                 const float2 scale2 = make_float2(scale, scale);
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                        static_cast<uint32_t>(b * BN + wg * HALF);

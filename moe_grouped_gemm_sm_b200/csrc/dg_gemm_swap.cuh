@@ -63,7 +63,8 @@ struct SwapLayout {
     static constexpr int W_BYTES = 128 * BK;                 // weight tile: 128 rows x 128 B
     static constexpr int X_BYTES = TN * BK;                  // activation tile: TN rows x 128 B
     static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
-    static constexpr int NBUF = (512 / TN) > 4 ? 4 : (512 / TN);
+    static constexpr int NBUF = 512 / TN;                    // TMEM buffers of TN columns
+    static constexpr int KG = 1;                             // K blocks per commit (see the MMA issuer)
     static constexpr int SFS = 16;                           // A-scale ring (a power of two), own barriers
     static constexpr int OFF_W = 0;
     static constexpr int OFF_X = OFF_W + STAGES * W_BYTES;
@@ -77,7 +78,7 @@ struct SwapLayout {
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int BYTES = OFF_MISC + static_cast<int>(sizeof(WaitCtx));
     static constexpr int ALLOC = BYTES + 1024;
-    static constexpr uint32_t TMEM_COLS = NBUF * TN <= 256 ? (NBUF * TN <= 128 ? 128 : 256) : 512;
+    static constexpr uint32_t TMEM_COLS = 512;
     static_assert(OFF_X % 1024 == 0 && OFF_SFA % 16 == 0 && OFF_C % 128 == 0, "aligned tiles");
     static_assert(ALLOC <= 232448, "shared memory budget");
 };
@@ -265,24 +266,31 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
         } else if (warp == 1 && lane == 0) {
             // ---------------- MMA issuer ----------------
             constexpr uint32_t IDESC = idesc_f8_e4m3_f32<128, TN>();
+            // one commit per K block (KG = 1): grouping commits, which saves tensor-pipe drains,
+            // measured slower here, where the run is bandwidth-bound and the tile tails matter
             uint32_t it = 0;
-            for (long long u = sk.u0; u < sk.u1 && !*abort_flag;) {
+            bool ok = true;
+            for (long long u = sk.u0; u < sk.u1 && ok;) {
                 int tile, kbs, kbe;
                 sk.segment(u, tile, kbs, kbe);
                 u += kbe - kbs;
+                int pending = 0;
                 for (int kb = kbs; kb < kbe; ++kb, ++it) {
                     const int s = it % STAGES;
                     const int b = it % NBUF;
-                    if (!mbar_wait(&full[s], (it / STAGES) & 1, ctx)) break;
-                    if (!mbar_wait(&tempty[b], ((it / NBUF) & 1) ^ 1, ctx)) break;
+                    ok = mbar_wait(&full[s], (it / STAGES) & 1, ctx) && mbar_wait(&tempty[b], ((it / NBUF) & 1) ^ 1, ctx);
+                    if (!ok) break;
                     tc_fence_after();
                     const uint64_t wd = sdesc_k_sw128(smem_u32(smem + L::OFF_W + s * L::W_BYTES));
                     const uint64_t xd = sdesc_k_sw128(smem_u32(smem + L::OFF_X + s * L::X_BYTES));
                     const uint32_t dt = tmem_base + static_cast<uint32_t>(b * TN);
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k) umma_f8(dt, wd + 2 * k, xd + 2 * k, IDESC, k > 0 ? 1u : 0u);
-                    umma_commit(&empty[s]);
-                    umma_commit(&tfull[b]);
+                    if (++pending == L::KG || kb + 1 == kbe) {
+                        for (uint32_t q = it + 1 - pending; q <= it; ++q) umma_commit(&empty[q % STAGES]);
+                        for (uint32_t q = it + 1 - pending; q <= it; ++q) umma_commit(&tfull[q % NBUF]);
+                        pending = 0;
+                    }
                 }
             }
         }
@@ -360,6 +368,7 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
             };
             auto release = [&](uint32_t itx) {
                 tc_fence_before();
+                fence_proxy_async_smem();   // A-scale reads before the slot's next TMA write
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive_relaxed(&sfa_empty[itx % L::SFS]);

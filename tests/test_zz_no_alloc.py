@@ -1,7 +1,16 @@
-"""dg_fp8_gemm_nt_noalloc: the few-row GEMM with the library's static scratch instead of the
-per-stream workspace. It must give exactly what dg_fp8_gemm_nt gives (same kernel, same work
-split), call after call (its flags are back to zero after every launch), allocate no device
-memory, work under CUDA-graph capture on a fresh stream, and refuse rows it cannot take."""
+"""dg_fp8_gemm_nt_noalloc: the stream-K few-row GEMM with the library's static scratch instead of
+the per-stream workspace. It must give exactly what dg_fp8_gemm_nt gives when that call takes
+the stream-K kernel too (same kernel, same work split), call after call (its flags are back to
+zero after every launch), allocate no device memory, work under CUDA-graph capture on a fresh
+stream, and refuse rows it cannot take.
+
+dg_fp8_gemm_nt picks its few-row kernel by shape; DG_FEW_ROW=streamk makes it always take the
+stream-K kernel. The library reads that variable once per process, so the tests that compare
+with dg_fp8_gemm_nt run in a child pytest process with it set."""
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -10,6 +19,18 @@ from moe_grouped_gemm_sm_b200 import _lib, build, ops, synth
 from tests.gpu_util import assert_close, bf16_dev, bf16_host_f64, host
 
 pytestmark = pytest.mark.gpu
+HERE = os.path.dirname(os.path.abspath(__file__))
+CHILD = os.environ.get("DG_FEW_ROW") == "streamk"
+child_only = pytest.mark.skipif(not CHILD, reason="runs in the DG_FEW_ROW=streamk child process")
+
+
+@pytest.mark.skipif(CHILD, reason="parent-process test")
+def test_in_a_streamk_child_process():
+    env = dict(os.environ, DG_FEW_ROW="streamk")
+    cmd = [sys.executable, "-m", "pytest", os.path.join(HERE, "test_zz_no_alloc.py"), "-q", "-x", "-m", "gpu"]
+    r = subprocess.run(cmd, cwd=os.path.dirname(HERE), env=env, capture_output=True, text=True, timeout=1200)
+    tail = "\n".join((r.stdout + r.stderr).splitlines()[-25:])
+    assert r.returncode == 0 and " passed" in r.stdout, tail
 
 SHAPES = [(1, 128, 128), (37, 264, 640), (64, 2112, 7168), (100, 1000, 896), (128, 4096, 7168)]
 
@@ -31,6 +52,7 @@ def sentinel(M, N):
     return torch.full((M, N), -3.0, dtype=torch.bfloat16, device="cuda")
 
 
+@child_only
 @pytest.mark.parametrize("M,N,K", SHAPES)
 @pytest.mark.parametrize("with_c", [False, True])
 def test_same_bits_as_the_allocating_entry_point_twice(M, N, K, with_c):
@@ -58,6 +80,7 @@ def test_matches_the_oracle(oracle):
     assert_close(bf16_host_f64(d), ref, "noalloc 64x2112x7168")
 
 
+@child_only
 def test_allocates_nothing_on_a_new_stream():
     M, N, K = 64, 2112, 7168
     (a, sfa, b, sfb, c), _ = operands(M, N, K, True, salt=6)
@@ -76,6 +99,7 @@ def test_allocates_nothing_on_a_new_stream():
     assert torch.cuda.mem_get_info()[0] < free0
 
 
+@child_only
 def test_graph_capture_on_a_fresh_stream_replays_exactly():
     M, N, K = 64, 2112, 7168
     (a, sfa, b, sfb, c), _ = operands(M, N, K, False, salt=7)
