@@ -315,6 +315,9 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
             const bool do_c = owner && p.has_c;
             if (do_c) {
                 // the previous tile's C has been read by every math thread before it is replaced
+                // by the next TMA write (each reader's proxy fence orders its generic reads
+                // before that async-proxy write)
+                fence_proxy_async_smem();
                 asm volatile("bar.sync 1, %0;" ::"n"(128 * L::NWG) : "memory");
                 if (threadIdx.x == 128 && ok) {
                     fence_proxy_async_smem();
