@@ -116,3 +116,33 @@ def test_prefill_shapes_sampled_rows(oracle, N, K):
         rows = rows[::2]
     ref = oracle.gemm_nt(*hv, rows=rows)
     assert_close(bf16_host_f64(d)[rows], ref, f"prefill 4096x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 2112, 7168), (128, 4096, 7168), (64, 24576, 1536)])
+def test_few_row_graph_capture_on_a_fresh_stream(oracle, M, N, K):
+    """A few-row GEMM captured into a CUDA graph on a stream that never ran one before. The
+    cluster split-K shapes (the first two) need no workspace and replay bit for bit what the
+    eager call gives. The stream-K shape cannot allocate its workspace under capture and takes
+    the tile kernel instead; it replays exactly and stays within the oracle's bound."""
+    dv, hv = quantised(oracle, M, N, K, True, salt=M + N)
+    eager = ops.fp8_gemm_nt(*dv)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    out = torch.full((M, N), -3.0, dtype=torch.bfloat16, device="cuda")
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        ops.fp8_gemm_nt(*dv, out=out, stream=s)
+    replays = []
+    for _ in range(3):
+        out.fill_(-3.0)
+        g.replay()
+        torch.cuda.synchronize()
+        replays.append(out.clone())
+    for r in replays[1:]:
+        assert torch.equal(r.view(torch.int16), replays[0].view(torch.int16))
+    cluster_shape = (N + 127) // 128 <= 64 and K // 128 <= 64
+    if cluster_shape:
+        assert torch.equal(replays[0].view(torch.int16), eager.view(torch.int16))
+    rows = sample_rows(M, extra=8) if N * K > 16 * 2 ** 20 else np.arange(M, dtype=np.int32)
+    ref = oracle.gemm_nt(*hv, rows=rows)
+    assert_close(bf16_host_f64(replays[0])[rows], ref, f"graph-captured {M}x{N}x{K}")
