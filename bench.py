@@ -223,6 +223,16 @@ def algorithmic_bytes(p):
     return V * K + 4 * V * kb + w + 2 * V * N + 4 * G
 
 
+def gemm_kernel_name(p):
+    """The library's kernel for a problem, by the library's documented dispatch rule (include/dg.h):
+    at most 128 rows per group (dense) take a few-row kernel, the cluster split-K one for at most
+    64 weight tiles and K <= 8192, stream-K otherwise; everything else the CTA-pair tile kernel."""
+    if p["kind"] == "dense" and p["rows"] <= 128:
+        small = (p["N"] + 127) // 128 <= 64 and p["K"] // 128 <= 64
+        return "gemm_splitk_kernel" if small else "gemm_swap_kernel"
+    return "gemm_kernel"
+
+
 def cast_bytes(p):
     """Per-token cast of all activation rows: 2 B read and 1 B written per element, plus scales."""
     rows = p["rows"] * (p["G"] if p["kind"] == "masked" else 1)
@@ -427,7 +437,7 @@ def run_cuda(args):
         t_tc = p["flops"] / (fp8_peak * 1e12)
         t_hbm = p["bytes"] / (hbm * 1e9)
         t_roof_total += max(t_tc, t_hbm)
-        per_problem.append({"N": p["N"], "K": p["K"], "gemm_us": round(gm * 1e3, 2),
+        per_problem.append({"N": p["N"], "K": p["K"], "kernel": gemm_kernel_name(p), "gemm_us": round(gm * 1e3, 2),
                             "tflops": round(p["flops"] / (gm * 1e-3) / 1e12, 1),
                             "gbs": round(p["bytes"] / (gm * 1e-3) / 1e9, 1),
                             "bound": "tensor" if t_tc >= t_hbm else "hbm",
@@ -448,7 +458,8 @@ def run_cuda(args):
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": round(hbm, 1), "unit": "GB/s",
                 "frac": round(achieved / hbm, 4), "peak_source": f"{peaks_src}: hbm_gbs (copy bandwidth)"}
     roof["roofline_time_frac"] = round(t_roof_total / gemm_total_s, 4)
-    roof["kernel"] = f"gemm_kernel ({len(probs)} problems, aggregate over launches)"
+    names = sorted({p["kernel"] for p in per_problem})
+    roof["kernel"] = f"{' + '.join(names)} ({len(probs)} problems, aggregate over launches)"
     roof["traffic"] = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
