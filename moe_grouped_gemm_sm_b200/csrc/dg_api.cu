@@ -188,14 +188,16 @@ bool use_streamk(int groups, int m_tiles, int N, int K) {
     return tiles > 64 || K / 128 > 64;
 }
 
-// Failure test only (DG_TEST_SKIP_RELEASE=1): the tile GEMM withholds one TMEM-buffer release,
-// so that a pipeline wait runs out of time and reports DG_ERR_TIMEOUT without faulting.
+// Failure tests only (DG_TEST_SKIP_RELEASE): 1 = the tile GEMM withholds one TMEM-buffer
+// release, 2 = the cluster split-K GEMM withholds one partial-push arrive. A bounded wait then
+// runs out of time and reports DG_ERR_TIMEOUT without faulting. 0 = off.
 int test_skip_release() {
     static std::atomic<int> cached{-1};
     int v = cached.load();
     if (v < 0) {
         const char *s = std::getenv("DG_TEST_SKIP_RELEASE");
-        v = s && std::atoi(s) ? 1 : 0;
+        v = s ? std::atoi(s) : 0;
+        if (v != 1 && v != 2) v = 0;
         cached.store(v);
     }
     return v;
@@ -350,7 +352,7 @@ dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.err = di->err;
     p.timeout_ns = wait_limit_ns();
-    p.test_skip_release = test_skip_release();
+    p.test_skip_release = test_skip_release() == 1;
     const bool batched = KIND == dg::KIND_MASKED;
     const int fbn = forced_bn();
     const int bn = fbn ? fbn : (N > 128 ? 256 : 128);
@@ -635,6 +637,7 @@ dg_status run_splitk(const void *a, const float *sfa, const void *b, const float
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.err = di->err;
     p.timeout_ns = wait_limit_ns();
+    p.test_skip_release = test_skip_release() == 2;
     // tiles the cluster count is sized for: the masked layout's real count depends on masked_m,
     // estimated from expected_m
     const int m_est = batched ? (hint + tn - 1) / tn : p.m_tiles;

@@ -413,7 +413,8 @@ __global__ void __launch_bounds__(SplitLayout<TN, STAGES>::THREADS, 1)
                 if (ok) {
 #pragma unroll
                     for (int e = 0; e < COLS; ++e) st_cluster_f32(push_addr + e * push_step, acc[e]);
-                    mbar_arrive_remote_release(push_bar);
+                    if (!(p.test_skip_release && blockIdx.x == 0 && warp == 4 && ti == 0))
+                        mbar_arrive_remote_release(push_bar);
                 }
                 if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait_cluster(recv_full, ti & 1, ctx));
             }

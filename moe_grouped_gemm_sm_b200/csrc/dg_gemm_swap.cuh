@@ -52,6 +52,7 @@ struct SwapParams {
     int *flags;       // [gridDim.x]; all zero between launches
     int *err;
     uint64_t timeout_ns;
+    int test_skip_release;   // failure test only (cluster kernel): CTA 0's warp 4 withholds its first push arrive
 };
 
 template <int TN, int STAGES>

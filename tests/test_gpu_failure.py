@@ -17,7 +17,8 @@ pytestmark = pytest.mark.gpu
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-CHILD = os.environ.get("DG_TEST_SKIP_RELEASE") == "1"
+MODE = os.environ.get("DG_TEST_SKIP_RELEASE", "")
+CHILD = MODE in ("1", "2")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -84,7 +85,44 @@ def test_pipeline_wait_timeout_is_reported():
     assert r.returncode == 0 and " passed" in r.stdout, tail
 
 
-@pytest.mark.skipif(not CHILD, reason="runs in the child process of test_pipeline_wait_timeout_is_reported")
+@pytest.mark.skipif(CHILD, reason="parent-process test")
+def test_cluster_exchange_wait_timeout_is_reported():
+    """A child process makes one math warp of the first cluster of the cluster split-K kernel
+    withhold its partial-push arrive (a debug-only switch), with a 100 ms wait limit: the reducers'
+    waits run out, every CTA of the cluster still meets the final cluster barrier and frees TMEM,
+    and DG_ERR_TIMEOUT is reported; the context then still computes correctly."""
+    env = dict(os.environ, DG_TEST_SKIP_RELEASE="2", DG_WAIT_TIMEOUT_MS="100", DG_FEW_ROW="cluster")
+    cmd = [sys.executable, "-m", "pytest", os.path.join(HERE, "test_gpu_failure.py"), "-q", "-x", "-m", "gpu",
+           "-k", "child"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    tail = "\n".join((r.stdout + r.stderr).splitlines()[-25:])
+    assert r.returncode == 0 and " passed" in r.stdout, tail
+
+
+@pytest.mark.skipif(MODE != "2", reason="runs in the child process of test_cluster_exchange_wait_timeout_is_reported")
+def test_child_cluster_timeout_then_recovery(oracle):
+    M, N, K = 64, 2112, 7168                              # 17 tiles: clusters of 6 CTAs
+    x, w, c = synth.dense_inputs(M, N, K, False, salt=43)
+    a, sfa = ops.cast_per_token(bf16_dev(x))
+    b, sfb = ops.cast_per_block(bf16_dev(w))
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+    ops.fp8_gemm_nt(a, sfa, b, sfb, None)
+    torch.cuda.synchronize()
+    assert _lib.dg_get_device_error() == _lib.DG_ERR_TIMEOUT
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+    # the context is usable: a many-row GEMM (the tile kernel, no withheld arrive) is exact
+    M2, N2, K2 = 512, 512, 1024
+    x2, w2, _ = synth.dense_inputs(M2, N2, K2, False, salt=44)
+    a2, sfa2 = ops.cast_per_token(bf16_dev(x2))
+    b2, sfb2 = ops.cast_per_block(bf16_dev(w2))
+    d2 = ops.fp8_gemm_nt(a2, sfa2, b2, sfb2, None)
+    torch.cuda.synchronize()
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+    ref = oracle.gemm_nt(host(a2), host(sfa2), host(b2), host(sfb2), None)
+    assert_close(bf16_host_f64(d2), ref, "after a cluster timeout")
+
+
+@pytest.mark.skipif(MODE != "1", reason="runs in the child process of test_pipeline_wait_timeout_is_reported")
 def test_child_timeout_then_recovery(oracle):
     M, N, K = 512, 512, 1024                              # CTA-pair tiles, several K blocks
     x, w, c = synth.dense_inputs(M, N, K, False, salt=41)
