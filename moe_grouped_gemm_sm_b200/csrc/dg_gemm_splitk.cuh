@@ -17,10 +17,11 @@
 //     reducer's mbarrier), so CTA j receives its rows [8·floor(16j/S), 8·floor(16(j+1)/S)) of
 //     all S partials, sums them in rank order (deterministic), adds C and writes D. No global
 //     workspace, no flags: the partials stay on chip;
-//   * one tcgen05.commit per K block. A commit drains the tensor pipe (four M=128 MMAs and their
-//     commit take ~830 cycles whatever N is, against ~360 per K block with one commit per four
-//     K blocks), but each SM streams a K block's 24-32 KB in ~1000 cycles here, so the MMA has
-//     the slack, and grouping commits only delays the promotion (measured slower).
+//   * one tcgen05.commit per K block. A commit drains the tensor pipe: four M=128 MMAs and their
+//     commit take ~830 cycles whatever N is, against ~355 per K block for N = 64 with one commit
+//     per four K blocks. But each SM streams a K block's 24-32 KB in ~1000 cycles here, so the
+//     MMA has the slack, and grouping commits (KG > 1) only delays the promotion (measured
+//     slower).
 //
 // CTA layout: warps 0, 2, 3 TMA producers (weights and activations on two threads each, the A
 // scales on four), warp 1 TMEM allocator + single-thread tcgen05.mma issuer (kind::f8f6f4,
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(SplitLayout<TN, STAGES>::THREADS, 1)
                 }
             }
         } else if (warp == 1 && lane == 0) {
-            // ---------------- MMA issuer: commits per group of KG K blocks ----------------
+            // ---------------- MMA issuer: a commit per KG K blocks and at each tile's end ----------------
             constexpr uint32_t IDESC = idesc_f8_e4m3_f32<128, TN>();
             uint32_t it = 0;
             bool ok = true;
