@@ -223,6 +223,19 @@ def algorithmic_bytes(p):
     return V * K + 4 * V * kb + w + 2 * V * N + 4 * G
 
 
+def fp8_tensor_peak(peaks, clocks):
+    """Dense fp8 peak (TFLOP/s) for the clocks a timed region ran at, and which figure it is:
+    2x the burst bf16 GEMM figure when the SM clock stayed at its maximum, 2x the sustained one
+    (taken under the power cap) when the power cap was active or the median clock sat below 95 %
+    of the maximum."""
+    mhz, top = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    capped = "sw_power_cap" in clocks.get("reasons", []) or (mhz is not None and bool(top) and mhz < 0.95 * top)
+    if capped:
+        return 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), \
+            "bf16_tflops_sustained (the power cap was active or the clock below max)"
+    return 2.0 * peaks["bf16_tflops"], "bf16_tflops (burst; the clock stayed at max)"
+
+
 def gemm_kernel_name(p):
     """The library's kernel for a problem, by the library's documented dispatch rule (include/dg.h):
     at most 128 rows per group (dense) take a few-row kernel, the cluster split-K one for at most
@@ -433,13 +446,9 @@ def run_cuda(args):
     # in a seconds-long loop under the power cap) when the power cap was active or the median
     # clock sat below 95 % of the maximum. Both fractions are reported.
     clocks = clk.summary()
-    capped = "sw_power_cap" in clocks["reasons"] or (
-        clocks["sm_mhz"] is not None and clocks["sm_max_mhz"] and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
+    fp8_peak, peak_kind = fp8_tensor_peak(peaks, clocks)
     fp8_peak_burst = 2.0 * peaks["bf16_tflops"]
     fp8_peak_sustained = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    fp8_peak = fp8_peak_sustained if capped else fp8_peak_burst
-    peak_kind = ("bf16_tflops_sustained (the power cap was active or the clock below max)" if capped
-                 else "bf16_tflops (burst; the clock stayed at max)")
     hbm = peaks["hbm_gbs"]
     per_problem = []
     t_roof_total = 0.0
