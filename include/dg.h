@@ -34,7 +34,17 @@
  *    and nothing throws across this ABI.
  *  - Preconditions of the GEMMs: K % 128 == 0, N % 8 == 0 (16-byte D rows), M >= 0.
  *    The results of the GEMMs satisfy |D - ref| <= 2^-7·|ref| + 1e-2·rms(ref) against the
- *    exact fp64 value of the same block-scaled operands.
+ *    exact fp64 value of the same block-scaled operands. Every GEMM is deterministic: the
+ *    same inputs give the same bits, call after call.
+ *  - Environment variables, each read once per process:
+ *      DG_WAIT_TIMEOUT_MS  the limit of every pipeline wait inside a kernel (default 4000);
+ *                          on expiry the kernel stops and DG_ERR_TIMEOUT is reported.
+ *    For experiments and tests only (they change which kernel runs, never the result beyond
+ *    the stated bound): DG_FORCE_PAIR=0|1 (CTA pairs for the tile GEMM), DG_FORCE_BN=128|256,
+ *    DG_FORCE_SWAP=0|1 (few-row kernels off for M <= 128, or on for the masked layout),
+ *    DG_FEW_ROW=streamk|cluster, DG_SPLITK_S=1|2|3|4|6|8|16 (cluster size). Debug only:
+ *    DG_TEST_SKIP_RELEASE=1|2 makes one kernel withhold one barrier arrive, so that a wait
+ *    runs out of time (failure tests).
  */
 #ifndef DG_H
 #define DG_H
@@ -81,8 +91,9 @@ DG_API dg_status dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, 
  * same result bit for bit as dg_fp8_gemm_nt whenever that call takes the stream-K kernel (the
  * same kernel and the same split of the work), but the kernel's scratch (the partial sums and
  * their flags) is a fixed static device array of the library instead of a per-stream
- * workspace, so the call never allocates and may be made under graph capture on any stream. That array is shared by all streams of a device: calls of this entry point must
- * not run concurrently on one device. The pages have no counterpart of this entry point.
+ * workspace, so the call never allocates and may be made under graph capture on any stream.
+ * That array is shared by all streams of a device: calls of this entry point must not run
+ * concurrently on one device. The pages have no counterpart of this entry point.
  * Errors: those of dg_fp8_gemm_nt, plus DG_ERR_UNSUPPORTED (nothing queued) when M > 128 or
  * when the device has more than 256 SMs (the array's capacity). */
 DG_API dg_status dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b, const float *sfb,
