@@ -2,7 +2,8 @@
 """Benchmark of the FP8 block-scaled NT GEMM hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
-                    [--workload prefill|decode64|decode128|contiguous|masked] [--only N,K]
+                    [--workload prefill|config1|decode64|decode128|contiguous|masked] [--only N,K]
+                    [--no-workloads] [--sub-steps S]
 
 One step = one pass of the hot path over the workload: for each problem of the workload, the
 per-token FP8 cast of its bf16 activations (1x128 scales written in the MN-major layout) and
@@ -13,7 +14,11 @@ synthetic recipe of moe_grouped_gemm_sm_b200.synth: A, B ~ N(0,1) and C ~ N(0,0.
 contiguous experts hold U{2048..6144} rows padded to 128; masked experts U{64..256} rows.
 
 The default workload (the one the headline number is quoted on) is the dense prefill set:
-M = 4096 with (N,K) in the six DeepSeek-V3 GEMM shapes and a C addend.
+M = 4096 with (N,K) in the six DeepSeek-V3 GEMM shapes and a C addend. The same JSON line then
+carries a "workloads" object with the other page configurations, each timed in its own region
+with its own roofline and per-problem times: the 64x2112x7168 decode shape with C = 0
+(config1), the M = 64 and M = 128 decode sets with the L2 flushed before every step (cold) and
+back to back (warm), the G = 8 contiguous and the G = 16 masked MoE sets.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a device synchronise,
 timed with CUDA events on the launching stream; the max over ranks is reported. When one step's
@@ -47,6 +52,8 @@ if ROOT not in sys.path:
 PREFILL_SHAPES = [(2112, 7168), (24576, 1536), (32768, 512), (7168, 16384), (4096, 7168), (7168, 2048)]
 GROUPED_SHAPES = [(4096, 7168), (7168, 2048)]
 WORKLOADS = {
+    "config1": dict(kind="dense", M=64, shapes=[(2112, 7168)], with_c=False,
+                    desc="dense FP8 NT GEMM, M=64, N=2112, K=7168, C = 0 (the pages' decode headline shape)"),
     "prefill": dict(kind="dense", M=4096, shapes=PREFILL_SHAPES, with_c=True,
                     desc="dense FP8 NT GEMM, M=4096, (N,K) in the six DeepSeek-V3 prefill shapes, C bf16"),
     "decode64": dict(kind="dense", M=64, shapes=PREFILL_SHAPES, with_c=True,
@@ -236,16 +243,6 @@ def fp8_tensor_peak(peaks, clocks):
     return 2.0 * peaks["bf16_tflops"], "bf16_tflops (burst; the clock stayed at max)"
 
 
-def gemm_kernel_name(p):
-    """The library's kernel for a problem, by the library's documented dispatch rule (include/dg.h):
-    at most 128 rows per group (dense) take a few-row kernel, the cluster split-K one for at most
-    64 weight tiles and K <= 8192, stream-K otherwise; everything else the CTA-pair tile kernel."""
-    if p["kind"] == "dense" and p["rows"] <= 128:
-        small = (p["N"] + 127) // 128 <= 64 and p["K"] // 128 <= 64
-        return "gemm_splitk_kernel" if small else "gemm_swap_kernel"
-    return "gemm_kernel"
-
-
 def cast_bytes(p):
     """Per-token cast of all activation rows: 2 B read and 1 B written per element, plus scales."""
     rows = p["rows"] * (p["G"] if p["kind"] == "masked" else 1)
@@ -255,6 +252,265 @@ def cast_bytes(p):
 # ------------------------------------------------------------------------------------------------
 # CUDA arm
 # ------------------------------------------------------------------------------------------------
+
+# The page configurations measured beside the headline, each in its own timed region:
+# (key in the "workloads" object, workload, L2 policy: "flush" = a 256 MB write at the start of
+# every step, "warm" = back-to-back steps, None = the default rule of the workload's size).
+SUB_WORKLOADS = [
+    ("config1", "config1", "flush"),
+    ("decode64_cold", "decode64", "flush"),
+    ("decode64_warm", "decode64", "warm"),
+    ("decode128_cold", "decode128", "flush"),
+    ("decode128_warm", "decode128", "warm"),
+    ("contiguous", "contiguous", None),
+    ("masked", "masked", None),
+]
+
+
+def source_digest():
+    """sha1 of the CUDA sources: the DRAM traffic stored under profiles/ holds for this digest."""
+    import glob
+    import hashlib
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "moe_grouped_gemm_sm_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    return h.hexdigest()
+
+
+def stored_traffic(workload):
+    """Per-launch DRAM bytes (read + write) of the workload's GEMM from profiles/traffic.json, or
+    None when none was taken or the kernels changed since (a different source digest)."""
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(tpath):
+        return None
+    with open(tpath) as f:
+        entry = json.load(f).get(workload)
+    if not isinstance(entry, dict) or entry.get("source_sha1") != source_digest():
+        return None
+    return entry.get("bytes_per_launch")
+
+
+class CudaArm:
+    """Device state of the CUDA arm: the library, the stream and the cast weights, which the
+    workloads that share a weight (same shape and seed) reuse."""
+
+    def __init__(self, device):
+        import torch
+
+        from moe_grouped_gemm_sm_b200 import _lib
+        self.torch, self._lib = torch, _lib
+        self.device = device
+        self.L = _lib.load()
+        self.stream = torch.cuda.current_stream(device)
+        self.weights = {}
+
+    def bf16(self, bits):
+        import numpy as np
+        t = self.torch.from_numpy(np.ascontiguousarray(bits, np.uint16).view(np.int16))
+        return t.view(self.torch.bfloat16).to(self.device)
+
+    def prepare(self, wl):
+        """Device operands of every problem of a workload; the weights are cast once (offline,
+        as in inference) and that cast is timed on its own."""
+        import numpy as np
+        torch, dev = self.torch, self.device
+        from moe_grouped_gemm_sm_b200 import ops
+        probs = make_problems(wl)
+        wc_ms = []
+        for p in probs:
+            key = (p["kind"], p["salt"], p["N"], p["K"], p["G"])
+            if key not in self.weights:
+                w_dev = self.bf16(p["w"])
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                ops.cast_per_block(w_dev)                             # warm the weight cast once
+                e0.record(self.stream)
+                b, sfb = ops.cast_per_block(w_dev)
+                e1.record(self.stream)
+                torch.cuda.synchronize(dev)
+                nb, kb = (p["N"] + 127) // 128, p["K"] // 128
+                self.weights[key] = (b, sfb, e0.elapsed_time(e1), p["G"] * (3 * p["N"] * p["K"] + 4 * nb * kb))
+                del w_dev
+            p["b"], p["sfb"], t, nbytes = self.weights[key]
+            wc_ms.append((t, nbytes))
+            p["a"] = self.bf16(p["x"])
+            p["cd"] = self.bf16(p["c"]) if p["c"] is not None else None
+            batch = p["G"] if p["kind"] == "masked" else 1
+            p["batch"] = batch
+            p["aq"] = torch.empty(p["a"].shape, dtype=torch.uint8, device=dev)
+            p["sfa"] = torch.empty((batch, p["K"] // 128, (p["rows"] + 3) // 4 * 4), dtype=torch.float32, device=dev)
+            dshape = (p["G"], p["rows"], p["N"]) if p["kind"] == "masked" else (p["rows"], p["N"])
+            p["d"] = torch.zeros(dshape, dtype=torch.bfloat16, device=dev)
+            if p["kind"] == "contiguous":
+                p["gl"] = torch.from_numpy(p["layout"]).to(dev)
+            if p["kind"] == "masked":
+                p["mm"] = torch.from_numpy(p["masked_m"]).to(dev)
+        torch.cuda.synchronize(dev)
+        return probs, wc_ms
+
+    # ---- launches through the C ABI (the same calls a user makes) ----
+    def launch_cast(self, p, sptr):
+        rc = self.L.dg_cast_fp8_per_token(p["a"].data_ptr(), p["aq"].data_ptr(), p["sfa"].data_ptr(), p["batch"],
+                                          p["rows"], p["K"], sptr)
+        if rc:
+            raise self._lib.DgError("dg_cast_fp8_per_token", rc)
+
+    def launch_gemm(self, p, sptr):
+        L = self.L
+
+        def ptr(t):
+            return t.data_ptr() if t is not None else None
+        if p["kind"] == "dense":
+            rc = L.dg_fp8_gemm_nt(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]), ptr(p["cd"]), ptr(p["d"]),
+                                  p["rows"], p["N"], p["K"], sptr)
+        elif p["kind"] == "contiguous":
+            rc = L.dg_m_grouped_fp8_gemm_nt_contiguous(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]),
+                                                       ptr(p["cd"]), ptr(p["d"]), ptr(p["gl"]), p["rows"], p["N"],
+                                                       p["K"], p["G"], sptr)
+        else:
+            rc = L.dg_m_grouped_fp8_gemm_nt_masked(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]),
+                                                   ptr(p["cd"]), ptr(p["d"]), ptr(p["mm"]), p["expected_m"], p["G"],
+                                                   p["rows"], p["N"], p["K"], sptr)
+        if rc:
+            raise self._lib.DgError("gemm", rc)
+
+    def time_steps(self, probs, steps, warmup, l2, local_rank):
+        """Times `steps` steps (per-token cast + GEMM per problem) as replays of one CUDA graph,
+        with CUDA events on the launching stream, clocks sampled during the region; then the
+        per-kernel durations from a second graph with an event pair around every launch."""
+        torch, dev = self.torch, self.device
+        stream = self.stream
+        step_bytes = sum(p["bytes"] + cast_bytes(p) for p in probs)
+        if l2 is None:
+            l2 = "flush" if step_bytes < 512 * 2 ** 20 else "large"
+        flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev) if l2 == "flush" else None
+
+        def step(sptr, ev=None):
+            if flush is not None:
+                flush.fill_(1)
+            cur = torch.cuda.current_stream(dev)
+            for i, p in enumerate(probs):
+                if ev is not None:
+                    ev[3 * i].record(cur)
+                self.launch_cast(p, sptr)
+                if ev is not None:
+                    ev[3 * i + 1].record(cur)
+                self.launch_gemm(p, sptr)
+                if ev is not None:
+                    ev[3 * i + 2].record(cur)
+
+        # eager warm-up, which also names the kernel each problem takes
+        for p in probs:
+            self.launch_cast(p, stream.cuda_stream)
+            self.launch_gemm(p, stream.cuda_stream)
+            p["kernel"] = self._lib.dg_last_kernel()
+        for _ in range(warmup):
+            step(stream.cuda_stream)
+        torch.cuda.synchronize(dev)
+        if self._lib.dg_get_device_error(stream.cuda_stream) != 0:
+            raise RuntimeError("device error word set during warm-up")
+
+        # The timed steps replay CUDA graphs (launch-bound decode steps would otherwise measure the
+        # host): `g_step` holds one step; `g_ev` the same step with an event pair around every
+        # launch, replayed separately for the per-kernel durations.
+        cap = torch.cuda.Stream(dev)
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3 * len(probs))]
+        g_step, g_ev = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            step(cap.cuda_stream)                                 # warm the capture stream
+            torch.cuda.synchronize(dev)
+            with torch.cuda.graph(g_step, stream=cap):
+                step(cap.cuda_stream)
+            with torch.cuda.graph(g_ev, stream=cap):
+                step(cap.cuda_stream, evs)
+        torch.cuda.synchronize(dev)
+        for _ in range(warmup):
+            g_step.replay()
+        torch.cuda.synchronize(dev)
+
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        with ClockSampler(local_rank) as clk:
+            start.record(stream)
+            for _ in range(steps):
+                g_step.replay()
+            end.record(stream)
+            torch.cuda.synchronize(dev)
+        barrier(dev)
+        local_ms = start.elapsed_time(end) / steps
+        if self._lib.dg_get_device_error(stream.cuda_stream) != 0:
+            raise RuntimeError("device error word set during the timed region")
+        cast_t = [[] for _ in probs]
+        gemm_t = [[] for _ in probs]
+        for _ in range(min(steps, 50)):
+            g_ev.replay()
+            torch.cuda.synchronize(dev)
+            for i in range(len(probs)):
+                cast_t[i].append(evs[3 * i].elapsed_time(evs[3 * i + 1]))
+                gemm_t[i].append(evs[3 * i + 1].elapsed_time(evs[3 * i + 2]))
+        del g_step, g_ev
+        return dict(local_ms=local_ms, cast_ms=[statistics.fmean(v) for v in cast_t],
+                    gemm_ms=[statistics.fmean(v) for v in gemm_t], clocks=clk.summary(), l2=l2,
+                    launches_per_step=2 * len(probs) + (1 if flush is not None else 0))
+
+
+L2_TEXT = {"flush": "256 MB L2-flushing write at the start of every step (cold weights)",
+           "warm": "no flush: steps back to back (weights partly L2-resident)",
+           "large": "no flush: one step's working set is far above the 126 MB L2"}
+
+
+def roofline_of(probs, t, workload):
+    """Roofline of the dominant kernel (the GEMM) over a workload's launches, and per problem."""
+    peaks, peaks_src = load_peaks()
+    # fp8 dense = 2 x bf16 (nominal ratio). The denominator matches the clocks the timed region
+    # ran at: the burst figure when the SM clock stayed at its maximum, the sustained one (taken
+    # in a seconds-long loop under the power cap) when the power cap was active or the median
+    # clock sat below 95 % of the maximum. Both fractions are reported.
+    fp8_peak, peak_kind = fp8_tensor_peak(peaks, t["clocks"])
+    fp8_peak_burst = 2.0 * peaks["bf16_tflops"]
+    fp8_peak_sustained = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    hbm = peaks["hbm_gbs"]
+    per_problem = []
+    t_roof_total = 0.0
+    for p, gm, cm in zip(probs, t["gemm_ms"], t["cast_ms"]):
+        t_tc = p["flops"] / (fp8_peak * 1e12)
+        t_hbm = p["bytes"] / (hbm * 1e9)
+        t_roof_total += max(t_tc, t_hbm)
+        per_problem.append({"N": p["N"], "K": p["K"], "rows": p["rows"], "G": p["G"],
+                            "kernel": p.get("kernel", ""), "flops": p["flops"], "bytes": p["bytes"],
+                            "gemm_us": round(gm * 1e3, 2),
+                            "tflops": round(p["flops"] / (gm * 1e-3) / 1e12, 1),
+                            "gbs": round(p["bytes"] / (gm * 1e-3) / 1e9, 1),
+                            "bound": "tensor" if t_tc >= t_hbm else "hbm",
+                            "roof_frac": round(max(t_tc, t_hbm) / (gm * 1e-3), 3),
+                            "cast_us": round(cm * 1e3, 2),
+                            "cast_gbs": round(cast_bytes(p) / (cm * 1e-3) / 1e9, 1)})
+    gemm_total_s = sum(t["gemm_ms"]) * 1e-3
+    flops_sum = sum(p["flops"] for p in probs)
+    bytes_sum = sum(p["bytes"] for p in probs)
+    if flops_sum / (fp8_peak * 1e12) >= bytes_sum / (hbm * 1e9):
+        achieved = flops_sum / gemm_total_s / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / fp8_peak, 4),
+                "peak_source": f"{peaks_src}: 2 x {peak_kind}; fp8 = 2x bf16 nominal ratio",
+                "frac_of_burst_peak": round(achieved / fp8_peak_burst, 4),
+                "frac_of_sustained_peak": round(achieved / fp8_peak_sustained, 4)}
+    else:
+        achieved = bytes_sum / gemm_total_s / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": round(hbm, 1), "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "peak_source": f"{peaks_src}: hbm_gbs (copy bandwidth)"}
+    roof["roofline_time_frac"] = round(t_roof_total / gemm_total_s, 4)
+    names = sorted({p["kernel"] for p in per_problem})
+    roof["kernel"] = f"{' + '.join(names)} ({len(probs)} problems, aggregate over launches)"
+    roof["timing"] = ("per-kernel CUDA events from a second graph with an event pair around every launch; the "
+                      "pairs stop the GEMM's prologue from overlapping the cast (programmatic dependent launch), "
+                      "so achieved slightly understates the GEMM")
+    roof["traffic"] = stored_traffic(workload)
+    return roof, per_problem
+
 
 def run_cuda(args):
     import numpy as np
@@ -269,136 +525,14 @@ def run_cuda(args):
     if world > 1:
         dist_init("nccl")
     _build.build()
-    L = _lib.load()
+    arm = CudaArm(device)
+    stream = arm.stream
     wl = WORKLOADS[args.workload]
-    stream = torch.cuda.current_stream(device)
-    sptr = stream.cuda_stream
 
-    def bf16(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits, np.uint16).view(np.int16)).view(torch.bfloat16).to(device)
-
-    probs = make_problems(wl)
-    wc_ms = []
-    for p in probs:
-        w_dev = bf16(p["w"])
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ops.cast_per_block(w_dev)                             # warm the weight cast once
-        e0.record(stream)
-        p["b"], p["sfb"] = ops.cast_per_block(w_dev)
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        nb, kb = (p["N"] + 127) // 128, p["K"] // 128
-        wc_ms.append((e0.elapsed_time(e1), p["G"] * (3 * p["N"] * p["K"] + 4 * nb * kb)))
-        del w_dev
-        p["a"] = bf16(p["x"])
-        p["cd"] = bf16(p["c"]) if p["c"] is not None else None
-        batch = p["G"] if p["kind"] == "masked" else 1
-        p["batch"] = batch
-        p["aq"] = torch.empty(p["a"].shape, dtype=torch.uint8, device=device)
-        p["sfa"] = torch.empty((batch, p["K"] // 128, (p["rows"] + 3) // 4 * 4), dtype=torch.float32, device=device)
-        dshape = (p["G"], p["rows"], p["N"]) if p["kind"] == "masked" else (p["rows"], p["N"])
-        p["d"] = torch.zeros(dshape, dtype=torch.bfloat16, device=device)
-        if p["kind"] == "contiguous":
-            p["gl"] = torch.from_numpy(p["layout"]).to(device)
-        if p["kind"] == "masked":
-            p["mm"] = torch.from_numpy(p["masked_m"]).to(device)
-    torch.cuda.synchronize(device)
-
-    def ptr(t):
-        return t.data_ptr() if t is not None else None
-
-    def launch_cast(p):
-        rc = L.dg_cast_fp8_per_token(ptr(p["a"]), ptr(p["aq"]), ptr(p["sfa"]), p["batch"], p["rows"], p["K"], sptr)
-        if rc:
-            raise _lib.DgError("dg_cast_fp8_per_token", rc)
-
-    def launch_gemm(p):
-        if p["kind"] == "dense":
-            rc = L.dg_fp8_gemm_nt(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]), ptr(p["cd"]), ptr(p["d"]),
-                                  p["rows"], p["N"], p["K"], sptr)
-        elif p["kind"] == "contiguous":
-            rc = L.dg_m_grouped_fp8_gemm_nt_contiguous(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]),
-                                                       ptr(p["cd"]), ptr(p["d"]), ptr(p["gl"]), p["rows"], p["N"],
-                                                       p["K"], p["G"], sptr)
-        else:
-            rc = L.dg_m_grouped_fp8_gemm_nt_masked(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]),
-                                                   ptr(p["cd"]), ptr(p["d"]), ptr(p["mm"]), p["expected_m"], p["G"],
-                                                   p["rows"], p["N"], p["K"], sptr)
-        if rc:
-            raise _lib.DgError("gemm", rc)
-
-    # small working sets (decode) fit in L2: flush it at the start of every step
-    step_bytes = sum(p["bytes"] + cast_bytes(p) for p in probs)
-    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=device) if step_bytes < 512 * 2 ** 20 else None
-
-    def step(ev=None):
-        if flush is not None:
-            flush.fill_(1)
-        cur = torch.cuda.current_stream(device)
-        for i, p in enumerate(probs):
-            if ev is not None:
-                ev[3 * i].record(cur)
-            launch_cast(p)
-            if ev is not None:
-                ev[3 * i + 1].record(cur)
-            launch_gemm(p)
-            if ev is not None:
-                ev[3 * i + 2].record(cur)
-
+    probs, wc_ms = arm.prepare(wl)
+    t = arm.time_steps(probs, args.steps, args.warmup, None, local_rank)
     flops_step = sum(p["flops"] for p in probs)
-    launches_per_step = 2 * len(probs) + (1 if flush is not None else 0)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(device)
-    if _lib.dg_get_device_error(sptr) != 0:
-        raise RuntimeError("device error word set during warm-up")
-
-    # The timed steps replay CUDA graphs (launch-bound decode steps would otherwise measure the
-    # host): `g_step` holds one step; `g_ev` the same step with an event pair around every
-    # launch, replayed separately for the per-kernel durations.
-    cap = torch.cuda.Stream(device)
-    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3 * len(probs))]
-    g_step, g_ev = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    cap.wait_stream(stream)
-    with torch.cuda.stream(cap):
-        sptr = cap.cuda_stream
-        step()                                            # warm the capture stream
-        torch.cuda.synchronize(device)
-        with torch.cuda.graph(g_step, stream=cap):
-            step()
-        with torch.cuda.graph(g_ev, stream=cap):
-            step(evs)
-    sptr = stream.cuda_stream
-    torch.cuda.synchronize(device)
-    for _ in range(args.warmup):
-        g_step.replay()
-    torch.cuda.synchronize(device)
-
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(device)
-    torch.cuda.synchronize(device)
-    with ClockSampler(local_rank) as clk:
-        start.record(stream)
-        for s in range(args.steps):
-            g_step.replay()
-        end.record(stream)
-        torch.cuda.synchronize(device)
-    barrier(device)
-    local_ms = start.elapsed_time(end) / args.steps
-    if _lib.dg_get_device_error(sptr) != 0:
-        raise RuntimeError("device error word set during the timed region")
-    cast_t = [[] for _ in probs]
-    gemm_t = [[] for _ in probs]
-    for _ in range(min(args.steps, 50)):
-        g_ev.replay()
-        torch.cuda.synchronize(device)
-        for i in range(len(probs)):
-            cast_t[i].append(evs[3 * i].elapsed_time(evs[3 * i + 1]))
-            gemm_t[i].append(evs[3 * i + 1].elapsed_time(evs[3 * i + 2]))
-    cast_ms = [statistics.fmean(v) for v in cast_t]
-    gemm_ms = [statistics.fmean(v) for v in gemm_t]
-    ms_max, flops_all = aggregate(local_ms, flops_step, device)
+    ms_max, flops_all = aggregate(t["local_ms"], flops_step, device)
     value = flops_all / (ms_max * 1e-3) / 1e12
 
     # ---------------- e2e through the public API with pinned host buffers ----------------
@@ -439,53 +573,8 @@ def run_cuda(args):
     e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, device)
     e2e_value = flops_all / (e2e_ms * 1e-3) / 1e12
 
-    # ---------------- roofline of the dominant kernel (the GEMM) ----------------
-    peaks, peaks_src = load_peaks()
-    # fp8 dense = 2 x bf16 (nominal ratio). The denominator matches the clocks the timed region
-    # ran at: the burst figure when the SM clock stayed at its maximum, the sustained one (taken
-    # in a seconds-long loop under the power cap) when the power cap was active or the median
-    # clock sat below 95 % of the maximum. Both fractions are reported.
-    clocks = clk.summary()
-    fp8_peak, peak_kind = fp8_tensor_peak(peaks, clocks)
-    fp8_peak_burst = 2.0 * peaks["bf16_tflops"]
-    fp8_peak_sustained = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    hbm = peaks["hbm_gbs"]
-    per_problem = []
-    t_roof_total = 0.0
-    for p, gm, cm in zip(probs, gemm_ms, cast_ms):
-        t_tc = p["flops"] / (fp8_peak * 1e12)
-        t_hbm = p["bytes"] / (hbm * 1e9)
-        t_roof_total += max(t_tc, t_hbm)
-        per_problem.append({"N": p["N"], "K": p["K"], "kernel": gemm_kernel_name(p), "gemm_us": round(gm * 1e3, 2),
-                            "tflops": round(p["flops"] / (gm * 1e-3) / 1e12, 1),
-                            "gbs": round(p["bytes"] / (gm * 1e-3) / 1e9, 1),
-                            "bound": "tensor" if t_tc >= t_hbm else "hbm",
-                            "roof_frac": round(max(t_tc, t_hbm) / (gm * 1e-3), 3),
-                            "cast_us": round(cm * 1e3, 2),
-                            "cast_gbs": round(cast_bytes(p) / (cm * 1e-3) / 1e9, 1)})
-    gemm_total_s = sum(gemm_ms) * 1e-3
-    flops_sum = sum(p["flops"] for p in probs)
-    bytes_sum = sum(p["bytes"] for p in probs)
-    if flops_sum / (fp8_peak * 1e12) >= bytes_sum / (hbm * 1e9):
-        achieved = flops_sum / gemm_total_s / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
-                "frac": round(achieved / fp8_peak, 4),
-                "peak_source": f"{peaks_src}: 2 x {peak_kind}; fp8 = 2x bf16 nominal ratio",
-                "frac_of_burst_peak": round(achieved / fp8_peak_burst, 4),
-                "frac_of_sustained_peak": round(achieved / fp8_peak_sustained, 4)}
-    else:
-        achieved = bytes_sum / gemm_total_s / 1e9
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": round(hbm, 1), "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "peak_source": f"{peaks_src}: hbm_gbs (copy bandwidth)"}
-    roof["roofline_time_frac"] = round(t_roof_total / gemm_total_s, 4)
-    names = sorted({p["kernel"] for p in per_problem})
-    roof["kernel"] = f"{' + '.join(names)} ({len(probs)} problems, aggregate over launches)"
-    roof["traffic"] = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            roof["traffic"] = json.load(f).get(args.workload)
-
+    roof, per_problem = roofline_of(probs, t, args.workload)
+    clocks = t["clocks"]
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
@@ -493,21 +582,47 @@ def run_cuda(args):
         "config": {"workload": wl["desc"], "shapes_NK": [list(s) for s in wl["shapes"]],
                    "step": "per-token cast of A + GEMM per problem; weights cast offline",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": ("256 MB flush at the start of every step" if flush is not None
-                          else "no flush: one step's working set is far above the 126 MB L2")},
+                   "l2": L2_TEXT[t["l2"]]},
         "roofline": roof,
         "per_problem": per_problem,
-        "weight_cast": {"gbs": round(sum(b for _, b in wc_ms) / (sum(t for t, _ in wc_ms) * 1e-3) / 1e9, 1),
-                        "ms_total": round(sum(t for t, _ in wc_ms), 3)},
+        "weight_cast": {"gbs": round(sum(b for _, b in wc_ms) / (sum(x for x, _ in wc_ms) * 1e-3) / 1e9, 1),
+                        "ms_total": round(sum(x for x, _ in wc_ms), 3)},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
                 "path": "pinned host activations (and C) -> device, ops cast + GEMM, D -> pinned host"},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": t["launches_per_step"] * args.steps,
         "launch": "each step replays a CUDA graph of its launches",
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, probs, target_s=args.cpu_seconds)
+    for p in probs:
+        p.clear()
+    del probs
+    arm.weights.clear()
+    torch.cuda.empty_cache()
+
+    # ---------------- the other page configurations, each in its own timed region ----------------
+    if not args.no_workloads and not args.only:
+        subs = {}
+        for key, name, l2 in SUB_WORKLOADS:
+            swl = WORKLOADS[name]
+            sprobs, _ = arm.prepare(swl)
+            st = arm.time_steps(sprobs, args.sub_steps, 3, l2, local_rank)
+            sms, sflops = aggregate(st["local_ms"], sum(p["flops"] for p in sprobs), device)
+            sroof, spp = roofline_of(sprobs, st, name if l2 != "warm" else key)
+            subs[key] = {"workload": swl["desc"], "value": round(sflops / (sms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                         "ms_per_step": round(sms, 4), "steps": args.sub_steps, "l2": L2_TEXT[st["l2"]],
+                         "gpu_launches": st["launches_per_step"] * args.sub_steps,
+                         "roofline": sroof, "per_problem": spp, "clocks": st["clocks"]}
+            for p in sprobs:
+                p.clear()
+            del sprobs
+            if name != "decode64":                              # decode128 reuses decode64's weights
+                arm.weights.clear()
+            torch.cuda.empty_cache()
+        result["workloads"] = subs
+
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -609,6 +724,10 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other page configurations (the 'workloads' object)")
+    ap.add_argument("--sub-steps", type=int, default=30,
+                    help="timed steps of each of the other page configurations")
     a = ap.parse_args(argv)
     a.warmup = max(3, a.warmup)          # at least three untimed warm-up steps
     return a

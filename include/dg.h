@@ -43,8 +43,8 @@
  *    the stated bound): DG_FORCE_PAIR=0|1 (CTA pairs for the tile GEMM), DG_FORCE_BN=128|256,
  *    DG_FORCE_SWAP=0|1 (few-row kernels off for M <= 128, or on for the masked layout),
  *    DG_FEW_ROW=streamk|cluster, DG_SPLITK_S=1|2|3|4|6|8|16 (cluster size). Debug only:
- *    DG_TEST_SKIP_RELEASE=1|2 makes one kernel withhold one barrier arrive, so that a wait
- *    runs out of time (failure tests).
+ *    DG_TEST_SKIP_RELEASE=1|2|3 makes one kernel withhold barrier arrives or partial flags,
+ *    so that a wait runs out of time (failure tests).
  */
 #ifndef DG_H
 #define DG_H
@@ -87,13 +87,20 @@ typedef enum dg_status {
 DG_API dg_status dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const float *sfb,
                          const void *c, void *d, int M, int N, int K, void *stream);
 
-/* dg_fp8_gemm_nt's stream-K path for M <= 128 without any allocation. Same arguments, and the
- * same result bit for bit as dg_fp8_gemm_nt whenever that call takes the stream-K kernel (the
- * same kernel and the same split of the work), but the kernel's scratch (the partial sums and
- * their flags) is a fixed static device array of the library instead of a per-stream
- * workspace, so the call never allocates and may be made under graph capture on any stream.
- * That array is shared by all streams of a device: calls of this entry point must not run
- * concurrently on one device. The pages have no counterpart of this entry point.
+/* dg_fp8_gemm_nt's stream-K path for M <= 128 without any allocation, for callers that must
+ * not call cudaMalloc (an allocator-owning runtime, a pre-planned memory arena, a decode loop
+ * that must not add allocations). Same arguments, and the same result bit for bit as
+ * dg_fp8_gemm_nt whenever that call takes the stream-K kernel (the same kernel and the same
+ * split of the work), but the kernel's scratch (the fp32 partial sums, their flags and a launch
+ * epoch) is a fixed static __device__ array of the library, 16 MB + 1 KB, instead of a
+ * per-stream workspace; every GPU that loads the library holds it until the process exits.
+ * The first call of any entry point on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before any stream
+ * capture. The array is shared by every call on a device and keeps what the last call left:
+ * calls that overlap on the GPU (on different streams, or replays of captured graphs that run
+ * at the same time) race on it and must not be made. Flags left by a launch that stopped early
+ * (after DG_ERR_TIMEOUT) are never taken for a later launch's: each launch waits for its own
+ * ticket. The pages have no counterpart of this entry point.
  * Errors: those of dg_fp8_gemm_nt, plus DG_ERR_UNSUPPORTED (nothing queued) when M > 128 or
  * when the device has more than 256 SMs (the array's capacity). */
 DG_API dg_status dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b, const float *sfb,
@@ -162,6 +169,15 @@ DG_API dg_status dg_get_device_error(void *stream);
 
 /* Static, human-readable name of a status code. */
 DG_API const char *dg_status_string(dg_status status);
+
+/* Name of the GEMM kernel that the calling thread's last GEMM call launched ("" before the
+ * first): "gemm_kernel", "gemm_kernel (CTA pairs)", "gemm_swap_kernel (stream-K)" or
+ * "gemm_splitk_kernel (cluster split-K)". For benchmarks and profiles; static storage. */
+DG_API const char *dg_last_kernel(void);
+
+/* Bytes of device memory the library has allocated with cudaMalloc so far, over all devices
+ * (the few-row stream-K workspaces); the static arrays of the module are not counted. */
+DG_API long long dg_allocated_bytes(void);
 
 #ifdef __cplusplus
 }

@@ -57,11 +57,14 @@ def load():
             "dg_sf_ld": [I],
             "dg_get_device_error": [P],
             "dg_status_string": [I],
+            "dg_last_kernel": [],
+            "dg_allocated_bytes": [],
         }
         for name, args in sig.items():
             f = getattr(L, name)
             f.argtypes = args
-            f.restype = ctypes.c_char_p if name == "dg_status_string" else I
+            f.restype = {"dg_status_string": ctypes.c_char_p, "dg_last_kernel": ctypes.c_char_p,
+                         "dg_allocated_bytes": ctypes.c_longlong}.get(name, I)
         _lib = L
     return _lib
 
@@ -131,3 +134,13 @@ def dg_get_device_error(stream=None) -> int:
 
 def dg_status_string(status: int) -> str:
     return load().dg_status_string(status).decode()
+
+
+def dg_last_kernel() -> str:
+    """Name of the GEMM kernel the calling thread's last GEMM call launched."""
+    return load().dg_last_kernel().decode()
+
+
+def dg_allocated_bytes() -> int:
+    """Device memory (bytes) the library has allocated with cudaMalloc so far."""
+    return int(load().dg_allocated_bytes())

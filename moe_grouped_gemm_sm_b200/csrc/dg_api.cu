@@ -25,13 +25,20 @@ constexpr int kMaxDevices = 64;
 __device__ int g_device_error;   // see dg_get_device_error()
 
 // Scratch of dg_fp8_gemm_nt_noalloc: the few-row kernel's stream-K partials and flags for up to
-// kStaticSlots CTAs, in the module's own device memory (zero-initialised at load).
+// kStaticSlots CTAs, then the two words of its launch epoch, in the module's own device memory
+// (zero-initialised at load).
 constexpr int kStaticSlots = 256;
 static __device__ __align__(256) float g_static_ws[kStaticSlots * 128 * 128];
-static __device__ __align__(256) int g_static_flags[kStaticSlots];
+static __device__ __align__(256) int g_static_flags[kStaticSlots + 2];
+
+// Device memory this library has allocated (cudaMalloc) so far, all devices; dg_allocated_bytes().
+std::atomic<long long> g_allocated{0};
+
+// Name of the GEMM kernel the calling thread's last GEMM call launched; dg_last_kernel().
+thread_local const char *t_last_kernel = "";
 
 struct DeviceInfo {
-    bool ready = false;
+    std::atomic<bool> ready{false};
     int sm_count = 0;
     int cc_major = 0, cc_minor = 0;
     int *err = nullptr;          // device address of g_device_error
@@ -50,9 +57,9 @@ dg_status device_info(const DeviceInfo **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DG_ERR_CUDA;
     DeviceInfo &d = g_dev[dev];
-    if (!d.ready) {
+    if (!d.ready.load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!d.ready) {
+        if (!d.ready.load(std::memory_order_relaxed)) {
             if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DG_ERR_CUDA;
             cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
             cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
@@ -68,7 +75,7 @@ dg_status device_info(const DeviceInfo **out) {
                     return DG_ERR_CUDA;
                 g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
             }
-            d.ready = true;
+            d.ready.store(true, std::memory_order_release);
         }
     }
     if (d.cc_major != 10 || d.cc_minor != 0) return DG_ERR_UNSUPPORTED;
@@ -189,18 +196,24 @@ bool use_streamk(int groups, int m_tiles, int N, int K) {
 }
 
 // Failure tests only (DG_TEST_SKIP_RELEASE): 1 = the tile GEMM withholds one TMEM-buffer
-// release, 2 = the cluster split-K GEMM withholds one partial-push arrive. A bounded wait then
-// runs out of time and reports DG_ERR_TIMEOUT without faulting. 0 = off.
+// release, 2 = the cluster split-K GEMM withholds one partial-push arrive, 3 = the process's
+// first two stream-K launches have their odd-numbered CTAs withhold their partial flags. A bounded wait
+// then runs out of time and reports DG_ERR_TIMEOUT without faulting. 0 = off.
 int test_skip_release() {
     static std::atomic<int> cached{-1};
     int v = cached.load();
     if (v < 0) {
         const char *s = std::getenv("DG_TEST_SKIP_RELEASE");
         v = s ? std::atoi(s) : 0;
-        if (v != 1 && v != 2) v = 0;
+        if (v != 1 && v != 2 && v != 3) v = 0;
         cached.store(v);
     }
     return v;
+}
+
+bool test_skip_streamk_flags() {
+    static std::atomic<int> launches{0};
+    return test_skip_release() == 3 && launches.fetch_add(1) < 2;
 }
 
 // Encodes a tiled tensor map. dims/box are innermost first; strides (bytes) for dims 1..rank-1.
@@ -324,6 +337,7 @@ dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p, int tiles, co
     if (n_units <= 0) return DG_OK;
     cfg.gridDim = dim3(PAIR ? 2 * n_units : n_units, 1, 1);
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mp.a, mp.b, mp.sfa, mp.c, mp.d, p);
+    t_last_kernel = PAIR ? "gemm_kernel (CTA pairs)" : "gemm_kernel";
     return from_cuda(e);
 }
 
@@ -427,15 +441,16 @@ bool build_swap_maps(SwapMaps &mp, const void *a, const float *sfa, const void *
     return true;
 }
 
-// Stream-K workspace of the few-row kernel: fp32 partials [slots][128][128] and one flag per
-// slot, flags zero between launches. One per (device, stream), so that launches on different
-// streams never share flags; allocated on a stream's first few-row call, which must not be
-// under graph capture (the call then takes the tile kernel, which needs no workspace).
+// Stream-K workspace of the few-row kernel: fp32 partials [slots][128][128], one flag per
+// slot and the two words of the launch epoch (all zero when allocated). One per (device,
+// stream), so that launches on different streams never share flags; allocated on a stream's
+// first few-row call, which must not be under graph capture (the call then takes the tile
+// kernel, which needs no workspace).
 struct SwapWorkspace {
     int dev = -1;
     cudaStream_t stream = nullptr;
     float *ws = nullptr;
-    int *flags = nullptr;
+    int *flags = nullptr;   // [slots] flags, then the epoch words
     int slots = 0;
 };
 std::vector<SwapWorkspace> g_swap_ws;
@@ -454,23 +469,21 @@ bool swap_workspace(int dev, int sm_count, cudaStream_t st, SwapWorkspace *out) 
     w.stream = st;
     w.slots = sm_count;
     const size_t ws_bytes = static_cast<size_t>(sm_count) * 128 * 128 * sizeof(float);
+    const size_t flag_bytes = static_cast<size_t>(sm_count + 2) * sizeof(int);
     if (cudaMalloc(&w.ws, ws_bytes) != cudaSuccess) return false;
-    if (cudaMalloc(&w.flags, static_cast<size_t>(sm_count) * sizeof(int)) != cudaSuccess ||
-        cudaMemset(w.flags, 0, static_cast<size_t>(sm_count) * sizeof(int)) != cudaSuccess) {
+    if (cudaMalloc(&w.flags, flag_bytes) != cudaSuccess) {
         cudaFree(w.ws);
         return false;
     }
+    if (cudaMemset(w.flags, 0, flag_bytes) != cudaSuccess) {
+        cudaFree(w.ws);
+        cudaFree(w.flags);
+        return false;
+    }
+    g_allocated += static_cast<long long>(ws_bytes + flag_bytes);
     g_swap_ws.push_back(w);
     *out = w;
     return true;
-}
-
-// After a device error a launch may have stopped with flags still set: zero this device's.
-void reset_swap_flags(int dev, const DeviceInfo *di) {
-    std::lock_guard<std::mutex> lk(g_mu);
-    for (const SwapWorkspace &w : g_swap_ws)
-        if (w.dev == dev) cudaMemset(w.flags, 0, static_cast<size_t>(w.slots) * sizeof(int));
-    cudaMemset(di->static_flags, 0, kStaticSlots * sizeof(int));
 }
 
 template <int TN, int STAGES, int KIND>
@@ -495,14 +508,16 @@ dg_status launch_swap(const SwapMaps &mp, const dg::SwapParams &p, long long til
     const long long grid = units < di->sm_count ? units : di->sm_count;
     if (grid <= 0) return DG_OK;
     Launch ln(dim3(static_cast<unsigned>(grid), 1, 1), dim3(L::THREADS, 1, 1), L::ALLOC, st);
+    t_last_kernel = "gemm_swap_kernel (stream-K)";
     return from_cuda(cudaLaunchKernelEx(&ln.cfg, kern, mp.w, mp.x, mp.sfa, mp.c, p));
 }
 
-// The few-row GEMM with the given stream-K scratch (partials for >= sm_count slots, flags zero).
+// The few-row GEMM with the given stream-K scratch: partials for `slots` >= sm_count CTAs, then
+// `slots` flags followed by the two epoch words.
 template <int KIND>
 dg_status run_swap_with(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
                         const int32_t *masked_m, int expected_m, int rows, int N, int K, int G, cudaStream_t st,
-                        const DeviceInfo *di, float *ws, int *flags) {
+                        const DeviceInfo *di, float *ws, int *flags, int slots) {
     const bool batched = KIND == dg::KIND_MASKED;
     const int hint = batched ? (expected_m > 0 ? expected_m : rows) : rows;
     const int tn = hint <= 64 ? 64 : 128;
@@ -523,8 +538,10 @@ dg_status run_swap_with(const void *a, const float *sfa, const void *b, const fl
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.ws = ws;
     p.flags = flags;
+    p.epoch = reinterpret_cast<unsigned *>(flags + slots);
     p.err = di->err;
     p.timeout_ns = wait_limit_ns();
+    p.test_skip_release = test_skip_streamk_flags() ? 3 : 0;
     // the largest possible tile set: masked groups may use fewer
     const long long tiles = static_cast<long long>(batched ? G : 1) * p.m_tiles * p.n_tiles;
     SwapMaps mp;
@@ -545,7 +562,8 @@ dg_status run_swap(const void *a, const float *sfa, const void *b, const float *
     if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
     SwapWorkspace w;
     if (!swap_workspace(dev, di->sm_count, st, &w)) return DG_ERR_UNSUPPORTED;
-    return run_swap_with<KIND>(a, sfa, b, sfb, c, d, masked_m, expected_m, rows, N, K, G, st, di, w.ws, w.flags);
+    return run_swap_with<KIND>(a, sfa, b, sfb, c, d, masked_m, expected_m, rows, N, K, G, st, di, w.ws, w.flags,
+                               w.slots);
 }
 
 // ---- few-row GEMMs: cluster split-K (dg_gemm_splitk.cuh) ----
@@ -608,6 +626,7 @@ dg_status launch_splitk(const SwapMaps &mp, const dg::SwapParams &p, int tiles, 
     }
     if (best_s == 0) return DG_ERR_UNSUPPORTED;
     Launch ln(dim3(static_cast<unsigned>(best_c * best_s), 1, 1), dim3(L::THREADS, 1, 1), L::ALLOC, st, best_s, true);
+    t_last_kernel = "gemm_splitk_kernel (cluster split-K)";
     return from_cuda(cudaLaunchKernelEx(&ln.cfg, kern, mp.w, mp.x, mp.sfa, p));
 }
 
@@ -637,7 +656,7 @@ dg_status run_splitk(const void *a, const float *sfa, const void *b, const float
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.err = di->err;
     p.timeout_ns = wait_limit_ns();
-    p.test_skip_release = test_skip_release() == 2;
+    p.test_skip_release = test_skip_release() == 2 ? 2 : 0;
     // tiles the cluster count is sized for: the masked layout's real count depends on masked_m,
     // estimated from expected_m
     const int m_est = batched ? (hint + tn - 1) / tn : p.m_tiles;
@@ -694,7 +713,8 @@ dg_status dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b,
     if (s != DG_OK) return s;
     if (di->sm_count > kStaticSlots) return DG_ERR_UNSUPPORTED;
     return run_swap_with<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, 0, M, N, K, 1,
-                                         static_cast<cudaStream_t>(stream), di, di->static_ws, di->static_flags);
+                                         static_cast<cudaStream_t>(stream), di, di->static_ws, di->static_flags,
+                                         kStaticSlots);
 }
 
 dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
@@ -793,13 +813,15 @@ dg_status dg_get_device_error(void *stream) {
     if (v != 0) {
         const int zero = 0;
         if (cudaMemcpy(di->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return DG_ERR_CUDA;
-        int dev = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess) reset_swap_flags(dev, di);
     }
     if (v == dg::ERR_TIMEOUT) return DG_ERR_TIMEOUT;
     if (v != 0) return DG_ERR_DEVICE;
     return DG_OK;
 }
+
+const char *dg_last_kernel(void) { return t_last_kernel; }
+
+long long dg_allocated_bytes(void) { return g_allocated.load(); }
 
 const char *dg_status_string(dg_status status) {
     switch (status) {

@@ -19,8 +19,11 @@
 //     global workspace, and the owner, for which the tile is the last segment of its run,
 //     adds them to its own in CTA order (a fixed order: results are deterministic), adds C and
 //     writes D (bf16, round to nearest even). Flags in the workspace tell the owner when a
-//     partial is complete; the owner clears each flag it consumed, so the workspace is back
-//     to all-zero flags at the end of every launch (CUDA-graph replays stay valid);
+//     partial is complete. A flag holds the ticket of the launch that wrote it: every launch
+//     reads the workspace's epoch word at its start and uses epoch + 1 as its ticket, and the
+//     last CTA to finish stores that ticket back into the epoch word. A flag left over from an
+//     earlier launch (one whose owner gave up after a bounded wait, say) therefore never
+//     matches, no flag needs clearing, and CUDA-graph replays stay valid;
 //   * a deep TMA ring (5-8 stages of the 16 KB weight tile) keeps enough bytes in flight.
 //
 // CTA layout: warps 0, 2, 3 TMA producers (weights and activations on two threads each, the A
@@ -49,11 +52,20 @@ struct SwapParams {
     const __nv_bfloat16 *c;
     __nv_bfloat16 *d;
     float *ws;        // stream-K partials, [gridDim.x][TN][128] fp32
-    int *flags;       // [gridDim.x]; all zero between launches
+    int *flags;       // [gridDim.x] partial flags, each the ticket of the launch that wrote it
+    unsigned *epoch;  // [2]: the last finished launch's ticket, and the count of finished CTAs
     int *err;
     uint64_t timeout_ns;
-    int test_skip_release;   // failure test only (cluster kernel): CTA 0's warp 4 withholds its first push arrive
+    // failure tests only: 2 = the cluster kernel's CTA 0, warp 4 withholds its first push
+    // arrive; 3 = the stream-K kernel's odd-numbered CTAs withhold their partial flags
+    int test_skip_release;
 };
+
+// Ticket of a stream-K launch: one past the epoch word, never 0 (flags start out zero).
+__device__ __forceinline__ int streamk_ticket(const unsigned *epoch) {
+    const unsigned e = *reinterpret_cast<const volatile unsigned *>(epoch);
+    return static_cast<int>(e + 1u == 0u ? 1u : e + 1u);
+}
 
 template <int TN, int STAGES>
 struct SwapLayout {
@@ -208,6 +220,8 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
         tmem_relinquish();
     }
     pdl_wait();   // from here on global memory may be read and written
+    __shared__ int ticket_smem;
+    if (threadIdx.x == 0) ticket_smem = streamk_ticket(p.epoch);
     if (KIND == KIND_MASKED && blockIdx.x == 0 && threadIdx.x == 0) {
         for (int gg = 0; gg < p.G; ++gg)
             if (__ldg(p.masked_m + gg) > p.M) report_error(p.err, ERR_DATA);
@@ -216,6 +230,7 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = ctx->tmem_base;
+    const int ticket = ticket_smem;
     volatile int *abort_flag = &ctx->abort;
     const SwapTiles<TN, KIND> tiles(p);
     const StreamK sk(tiles.count, p.Kb, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x), L::MAX_PARTS);
@@ -446,14 +461,15 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
                     __threadfence();
                 }
                 ok = named_barrier_and(2, 128 * L::NWG, ok);
-                if (threadIdx.x == 128 && ok) flag_store_release(p.flags + c_self, 1);
+                if (threadIdx.x == 128 && ok && !(p.test_skip_release == 3 && (c_self & 1)))
+                    flag_store_release(p.flags + c_self, ticket);
                 continue;
             }
             if (kbe < p.Kb) {
                 // The tile's later K blocks are partials of CTAs c_self+1 .. j1 (at most
-                // MAX_PARTS). Their flags are waited for (and cleared for the next launch), the
-                // partials copied in bulk into the operand ring, idle now (this is the run's last
-                // segment and its MMAs are done), and added in CTA order.
+                // MAX_PARTS). Their flags are waited for (each must hold this launch's ticket),
+                // the partials copied in bulk into the operand ring, idle now (this is the run's
+                // last segment and its MMAs are done), and added in CTA order.
                 const int j1 = sk.cta_of(static_cast<long long>(tile) * p.Kb + p.Kb - 1);
                 const int nparts = j1 - c_self;
                 bool got = ok && nparts <= L::MAX_PARTS;
@@ -461,7 +477,7 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
                 if (threadIdx.x == 128 && got) {
                     const uint64_t t0 = globaltimer_ns();
                     for (int jj = c_self + 1; jj <= j1 && got; ++jj) {
-                        while (flag_load_acquire(p.flags + jj) == 0) {
+                        while (flag_load_acquire(p.flags + jj) != ticket) {
                             if (*abort_flag) {
                                 got = false;
                                 break;
@@ -473,7 +489,6 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
                                 break;
                             }
                         }
-                        if (got) p.flags[jj] = 0;
                     }
                     if (got) mbar_arrive_expect_tx(fix_full, static_cast<uint32_t>(nparts) * L::PART_BYTES);
                 }
@@ -519,6 +534,16 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem_base, L::TMEM_COLS);
+    }
+    if (threadIdx.x == 0) {
+        // the last CTA to finish publishes this launch's ticket as the epoch; the next launch
+        // on the stream reads it only after this grid has completed (griddepcontrol.wait)
+        __threadfence();
+        if (atomicAdd(p.epoch + 1, 1u) == gridDim.x - 1) {
+            p.epoch[1] = 0u;
+            p.epoch[0] = static_cast<unsigned>(ticket);
+            __threadfence();
+        }
     }
 #endif
 }

@@ -31,15 +31,35 @@ def test_missing_sustained_figure_falls_back_to_burst():
     assert bench.fp8_tensor_peak(peaks, {"sm_mhz": 1000, "sm_max_mhz": 1965, "reasons": []})[0] == 200.0
 
 
-def test_kernel_names_follow_the_dispatch_rule():
-    dense = lambda M, N, K: {"kind": "dense", "rows": M, "N": N, "K": K}
-    # at most 128 rows: cluster split-K for <= 64 weight tiles and K <= 8192, else stream-K
-    assert bench.gemm_kernel_name(dense(64, 2112, 7168)) == "gemm_splitk_kernel"
-    assert bench.gemm_kernel_name(dense(128, 8192, 8192)) == "gemm_splitk_kernel"
-    assert bench.gemm_kernel_name(dense(128, 8193, 8192)) == "gemm_swap_kernel"      # 65 tiles
-    assert bench.gemm_kernel_name(dense(64, 7168, 16384)) == "gemm_swap_kernel"      # Kb = 128
-    assert bench.gemm_kernel_name(dense(64, 24576, 1536)) == "gemm_swap_kernel"      # 192 tiles
-    # more rows, and the grouped layouts: the tile kernel
-    assert bench.gemm_kernel_name(dense(129, 2112, 7168)) == "gemm_kernel"
-    assert bench.gemm_kernel_name({"kind": "masked", "rows": 256, "N": 4096, "K": 7168}) == "gemm_kernel"
-    assert bench.gemm_kernel_name({"kind": "contiguous", "rows": 32768, "N": 4096, "K": 7168}) == "gemm_kernel"
+def test_every_page_configuration_is_measured():
+    """The headline (prefill) plus the workloads object cover every configuration of the pages:
+    the 64x2112x7168 C = 0 decode shape, decode M = 64 and 128 cold and warm, contiguous, masked."""
+    keys = {k for k, _, _ in bench.SUB_WORKLOADS}
+    assert keys == {"config1", "decode64_cold", "decode64_warm", "decode128_cold", "decode128_warm",
+                    "contiguous", "masked"}
+    c1 = bench.WORKLOADS["config1"]
+    assert c1["M"] == 64 and c1["shapes"] == [(2112, 7168)] and not c1["with_c"]
+    for name in ("decode64", "decode128"):
+        assert bench.WORKLOADS[name]["shapes"] == bench.PREFILL_SHAPES
+    assert bench.WORKLOADS["contiguous"]["G"] == 8 and bench.WORKLOADS["masked"]["G"] == 16
+
+
+def test_algorithmic_bytes_of_the_decode_headline_shape():
+    """64x2112x7168 with C = 0: A and B e4m3, their fp32 scales, D bf16 (15.9 MB)."""
+    p = {"kind": "dense", "rows": 64, "N": 2112, "K": 7168, "G": 1, "with_c": False}
+    kb, nb = 56, 17
+    assert bench.algorithmic_bytes(p) == 64 * 7168 + 4 * 64 * kb + 2112 * 7168 + 4 * nb * kb + 2 * 64 * 2112
+
+
+def test_stored_traffic_is_dropped_when_the_kernels_change(tmp_path, monkeypatch):
+    import json
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "source_digest", lambda: "f" * 40)     # the current kernels' digest
+    (prof / "traffic.json").write_text(json.dumps({
+        "prefill": {"bytes_per_launch": 123.0, "source_sha1": "f" * 40},
+        "decode64": {"bytes_per_launch": 7.0, "source_sha1": "0" * 40}}))
+    assert bench.stored_traffic("prefill") == 123.0
+    assert bench.stored_traffic("decode64") is None
+    assert bench.stored_traffic("masked") is None

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 MODE = os.environ.get("DG_TEST_SKIP_RELEASE", "")
-CHILD = MODE in ("1", "2")
+CHILD = MODE in ("1", "2", "3")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -143,3 +143,47 @@ def test_child_timeout_then_recovery(oracle):
     assert _lib.dg_get_device_error() == _lib.DG_OK
     ref = oracle.gemm_nt(host(a2), host(sfa2), host(b2), host(sfb2), None)
     assert_close(bf16_host_f64(d2), ref, "after a timeout")
+
+
+@pytest.mark.skipif(CHILD, reason="parent-process test")
+def test_streamk_flag_wait_timeout_leaves_no_stale_flags():
+    """A child process makes the odd-numbered CTAs of its first two stream-K launches withhold
+    their partial flags (a debug-only switch), with a 100 ms wait limit: the owners' flag waits
+    run out, leaving the flags of the partials they did not reach set. Without a
+    dg_get_device_error() call in between, the next stream-K launches on the same per-stream
+    workspace and on the static scratch of dg_fp8_gemm_nt_noalloc must still be exact."""
+    env = dict(os.environ, DG_TEST_SKIP_RELEASE="3", DG_WAIT_TIMEOUT_MS="100", DG_FEW_ROW="streamk")
+    cmd = [sys.executable, "-m", "pytest", os.path.join(HERE, "test_gpu_failure.py"), "-q", "-x", "-m", "gpu",
+           "-k", "child"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    tail = "\n".join((r.stdout + r.stderr).splitlines()[-25:])
+    assert r.returncode == 0 and " passed" in r.stdout, tail
+
+
+@pytest.mark.skipif(MODE != "3", reason="runs in the child process of test_streamk_flag_wait_timeout_leaves_no_stale_flags")
+def test_child_streamk_timeout_then_exact(oracle):
+    M, N, K = 64, 4096, 7168          # 32 weight tiles of 56 K blocks: 4-6 partials per tile
+    x, w, c = synth.dense_inputs(M, N, K, True, salt=45)
+    x_bad, _, _ = synth.dense_inputs(M, N, K, False, salt=46)
+    b, sfb = ops.cast_per_block(bf16_dev(w))
+    a, sfa = ops.cast_per_token(bf16_dev(x))
+    a_bad, sfa_bad = ops.cast_per_token(bf16_dev(x_bad))   # other partials, so stale ones would show
+    cd = bf16_dev(c)
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+
+    def out():
+        return torch.full((M, N), -3.0, dtype=torch.bfloat16, device="cuda")
+
+    # the two withholding launches: the per-stream workspace, then the static scratch
+    _lib.dg_fp8_gemm_nt(a_bad, sfa_bad, b, sfb, cd, out(), M, N, K)
+    _lib.dg_fp8_gemm_nt_noalloc(a_bad, sfa_bad, b, sfb, cd, out(), M, N, K)
+    # no dg_get_device_error() here: the next launches find the flags as the failed ones left them
+    d_ws, d_static = out(), out()
+    _lib.dg_fp8_gemm_nt(a, sfa, b, sfb, cd, d_ws, M, N, K)
+    _lib.dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, cd, d_static, M, N, K)
+    torch.cuda.synchronize()
+    assert _lib.dg_get_device_error() == _lib.DG_ERR_TIMEOUT
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+    ref = oracle.gemm_nt(host(a), host(sfa), host(b), host(sfb), c)
+    assert_close(bf16_host_f64(d_ws), ref, "stream-K after a flag timeout")
+    assert torch.equal(d_static.view(torch.int16), d_ws.view(torch.int16))

@@ -95,13 +95,16 @@ def sample_rows(M, per_tile=2, extra=16, seed=0):
 @pytest.mark.parametrize("M", [64, 128])
 @pytest.mark.parametrize("N,K", PAGE_SHAPES)
 def test_decode_shapes_full_compare(oracle, M, N, K):
+    """Every element of the twelve decode shapes (at most ~15 G multiply-adds of fp64 on the
+    host each). In the few-row kernels the token rows are the MMA's N columns, spread over
+    several math warps and, for the split kernels, over several SMs: a fault confined to some
+    token columns shows up only in a full compare."""
     with_c = not (M == 64 and (N, K) == (2112, 7168))      # the 64x2112x7168 case has C = 0
     dv, hv = quantised(oracle, M, N, K, with_c, salt=N + K + M)
     d = ops.fp8_gemm_nt(*dv)
     torch.cuda.synchronize()
-    rows = np.arange(M, dtype=np.int32) if N * K <= 16 * 2 ** 20 else sample_rows(M, extra=8)
-    ref = oracle.gemm_nt(*hv, rows=rows)
-    assert_close(bf16_host_f64(d)[rows], ref, f"decode {M}x{N}x{K}")
+    ref = oracle.gemm_nt(*hv)
+    assert_close(bf16_host_f64(d), ref, f"decode {M}x{N}x{K}")
 
 
 @pytest.mark.slow
@@ -111,7 +114,7 @@ def test_prefill_shapes_sampled_rows(oracle, N, K):
     dv, hv = quantised(oracle, M, N, K, True, salt=N + K)
     d = ops.fp8_gemm_nt(*dv)
     torch.cuda.synchronize()
-    rows = sample_rows(M, extra=16, seed=N)
+    rows = sample_rows(M, extra=16, seed=N * 7 + K)
     if N * K > 64 * 2 ** 20:
         rows = rows[::2]
     ref = oracle.gemm_nt(*hv, rows=rows)
@@ -143,6 +146,5 @@ def test_few_row_graph_capture_on_a_fresh_stream(oracle, M, N, K):
     cluster_shape = (N + 127) // 128 <= 64 and K // 128 <= 64
     if cluster_shape:
         assert torch.equal(replays[0].view(torch.int16), eager.view(torch.int16))
-    rows = sample_rows(M, extra=8) if N * K > 16 * 2 ** 20 else np.arange(M, dtype=np.int32)
-    ref = oracle.gemm_nt(*hv, rows=rows)
-    assert_close(bf16_host_f64(replays[0])[rows], ref, f"graph-captured {M}x{N}x{K}")
+    ref = oracle.gemm_nt(*hv)
+    assert_close(bf16_host_f64(replays[0]), ref, f"graph-captured {M}x{N}x{K}")

@@ -1,8 +1,10 @@
 """dg_fp8_gemm_nt_noalloc: the stream-K few-row GEMM with the library's static scratch instead of
 the per-stream workspace. It must give exactly what dg_fp8_gemm_nt gives when that call takes
-the stream-K kernel too (same kernel, same work split), call after call (its flags are back to
-zero after every launch), allocate no device memory, work under CUDA-graph capture on a fresh
-stream, and refuse rows it cannot take.
+the stream-K kernel too (same kernel, same work split), call after call (flags left set by an
+earlier launch never match a later launch's ticket), allocate no device memory, work under
+CUDA-graph capture on a fresh stream, and refuse rows it cannot take. Some callers cannot
+allocate at all: a runtime that owns every byte of device memory through its own arena, or a
+decode loop whose memory plan is fixed; this entry point serves them.
 
 dg_fp8_gemm_nt picks its few-row kernel by shape; DG_FEW_ROW=streamk makes it always take the
 stream-K kernel. The library reads that variable once per process, so the tests that compare
@@ -82,21 +84,26 @@ def test_matches_the_oracle(oracle):
 
 @child_only
 def test_allocates_nothing_on_a_new_stream():
+    """The library counts every byte it allocates (dg_allocated_bytes): a call on a stream that
+    never saw one leaves the count as it was, where dg_fp8_gemm_nt allocates that stream's
+    workspace."""
     M, N, K = 64, 2112, 7168
     (a, sfa, b, sfb, c), _ = operands(M, N, K, True, salt=6)
     d = sentinel(M, N)
     _lib.dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, c, d, M, N, K)   # kernel loaded, tensors ready
     torch.cuda.synchronize()
     s = torch.cuda.Stream()
-    free0 = torch.cuda.mem_get_info()[0]
+    before = _lib.dg_allocated_bytes()
+    torch_before = torch.cuda.memory_allocated()
     _lib.dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, c, d, M, N, K, stream=s)
     torch.cuda.synchronize()
-    assert torch.cuda.mem_get_info()[0] == free0
+    assert _lib.dg_allocated_bytes() == before
+    assert torch.cuda.memory_allocated() == torch_before
     # the allocating entry point does allocate its workspace for a new stream
     s2 = torch.cuda.Stream()
     _lib.dg_fp8_gemm_nt(a, sfa, b, sfb, c, d, M, N, K, stream=s2)
     torch.cuda.synchronize()
-    assert torch.cuda.mem_get_info()[0] < free0
+    assert _lib.dg_allocated_bytes() > before
 
 
 @child_only
