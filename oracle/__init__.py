@@ -49,8 +49,11 @@ def lib():
         L.dgo_gemm_nt.argtypes = [P, P, P, P, P, I, I, I, P, I, P]
         L.dgo_m_grouped_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, P]
         L.dgo_m_grouped_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
+        L.dgo_cast_per_channel.argtypes = [P, I, I, P, P]
+        L.dgo_k_grouped_tn.argtypes = [P, P, P, P, P, P, I, I, I, P]
         for f in ("dgo_cast_per_token", "dgo_cast_per_block", "dgo_transform_sf", "dgo_gemm_nt",
-                  "dgo_m_grouped_contiguous", "dgo_m_grouped_masked", "dgo_num_threads"):
+                  "dgo_m_grouped_contiguous", "dgo_m_grouped_masked", "dgo_num_threads",
+                  "dgo_cast_per_channel", "dgo_k_grouped_tn"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -176,3 +179,49 @@ def tolerance_ok(d: np.ndarray, ref: np.ndarray, rel: float = 2.0 ** -7, abs_rms
     err = np.abs(d - ref)
     ratio = float(np.max(err / np.maximum(bound, 1e-300))) if ref.size else 0.0
     return bool(np.all(err <= bound)), ratio
+
+
+def gemm_layout(a, sfa, b, sfb, layout: str, c=None, rows=None) -> np.ndarray:
+    """fp64 D for the dense block-scaled GEMM in the layouts the pages name ([likun] §一/§二:
+    fp8_gemm_{nt,nn,tn,tt}). The first letter is A's storage, the second B's:
+      A "n": [M,K] (K contiguous)    A "t": [K,M] (M contiguous)
+      B "t": [N,K] (K contiguous)    B "n": [K,N] (N contiguous)
+    so that D[m,n] = C[m,n] + sum_k A_log[m,k]·B_log[n,k] with the same scales in every layout
+    (sfa [Kb][pad4(M)] per 1x128 slice of A along K, sfb [Nb][Kb] per 128x128 block). Moving an
+    operand from MN-major to K-major storage is a transpose (data movement only), after which
+    the NT definition applies."""
+    layout = layout.lower()
+    assert layout in ("nt", "nn", "tn", "tt"), layout
+    a = np.asarray(a)
+    b = np.asarray(b)
+    a_k = np.ascontiguousarray(a.T) if layout[0] == "t" else a
+    b_k = np.ascontiguousarray(b.T) if layout[1] == "n" else b
+    return gemm_nt(a_k, sfa, b_k, sfb, c, rows=rows)
+
+
+def cast_per_channel(x_bf16: np.ndarray):
+    """x [T,C] bf16 bits (T % 128 == 0) -> (q [T,C] uint8, sf [T/128, pad4(C)] fp32): one scale
+    per channel per 128-token block (the recipe (1,1,128) of the K-grouped GEMM)."""
+    x = _c(x_bf16, np.uint16)
+    T, C = x.shape
+    q = np.empty((T, C), np.uint8)
+    sf = np.zeros((T // 128, pad4(C)), np.float32)
+    _check(lib().dgo_cast_per_channel(_p(x), T, C, _p(q), _p(sf)), "cast_per_channel")
+    return q, sf
+
+
+def k_grouped_tn(a, sfa, b, sfb, ks, c=None) -> np.ndarray:
+    """fp64 D [G,M,N] of the K-grouped TN GEMM: a [sum_K, M], b [sum_K, N] e4m3 codes,
+    sfa [sum_K/128, pad4(M)], sfb [sum_K/128, pad4(N)] fp32, ks [G] group sizes (multiples of
+    128), c fp32 [G,M,N] or None."""
+    a = _c(a, np.uint8); b = _c(b, np.uint8)
+    sfa = _c(sfa, np.float32); sfb = _c(sfb, np.float32); c = _c(c, np.float32)
+    ks = _c(ks, np.int32)
+    G = ks.shape[0]
+    M, N = a.shape[1], b.shape[1]
+    assert a.shape[0] == b.shape[0] == int(ks.sum()), (a.shape, b.shape, ks)
+    assert sfa.shape == (a.shape[0] // 128, pad4(M)) and sfb.shape == (b.shape[0] // 128, pad4(N))
+    out = np.empty((G, M, N), np.float64)
+    _check(lib().dgo_k_grouped_tn(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(ks), G, M, N, _p(out)),
+           "k_grouped_tn")
+    return out

@@ -283,6 +283,82 @@ int dgo_m_grouped_masked(const uint8_t *a, const float *sfa, const uint8_t *b, c
     return 0;
 }
 
+/* ---------------------------------------------------------------------------------------- */
+/* K-grouped GEMM for the MoE weight gradient ([likun] §一: k_grouped_fp8_gemm_tn, "MoE 反向";  */
+/* §二: k_grouped_fp8_gemm_tn_contiguous with ks_cpu and recipe (1,1,128)).                   */
+/* ---------------------------------------------------------------------------------------- */
+
+/* Per-channel cast along the outer dimension, the recipe (1,1,128) quantisation of a
+ * token-major tensor: x bf16 [T,C] (T tokens, C channels contiguous), T % 128 == 0. For every
+ * 128-token block tb and channel c: amax = max_{t in tb} |x[t,c]|, s = amax/448 (s = 1 when
+ * amax = 0), q[t,c] = e4m3_satrne(x[t,c] / s); sf fp32 [T/128][pad4(C)], sf[tb*pad4(C) + c] = s
+ * (padding entries untouched). The same readings as the per-token cast, on the transposed
+ * tensor. */
+int dgo_cast_per_channel(const uint16_t *x, int T, int C, uint8_t *q, float *sf) {
+    if (T < 0 || C < 0 || T % DGO_BLK) return -1;
+    int Tb = T / DGO_BLK, ld = pad4(C);
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int tb = 0; tb < Tb; tb++) {
+        for (int c = 0; c < C; c++) {
+            float amax = 0.0f;
+            for (int i = 0; i < DGO_BLK; i++) {
+                float v = fabsf(dgo_bf16_to_f32(x[((size_t)tb * DGO_BLK + i) * C + c]));
+                if (v > amax) amax = v;
+            }
+            float s = scale_from_amax(amax);
+            for (int i = 0; i < DGO_BLK; i++) {
+                size_t off = ((size_t)tb * DGO_BLK + i) * C + c;
+                q[off] = dgo_e4m3_encode_satrne(dgo_bf16_to_f32(x[off]) / s);
+            }
+            sf[(size_t)tb * ld + c] = s;
+        }
+    }
+    return 0;
+}
+
+/* K-grouped TN GEMM: the K dimension (tokens) is cut into G consecutive groups of ks[g] rows
+ * (each a multiple of 128); group g owns rows [k0_g, k0_g + ks[g]) of both operands.
+ *   a  e4m3 [sum_K, M] (M contiguous: "T", the transposed A);  sfa fp32 [sum_K/128][pad4(M)]
+ *   b  e4m3 [sum_K, N] (N contiguous: "N");                      sfb fp32 [sum_K/128][pad4(N)]
+ *   c  fp32 [G, M, N] or NULL;  out fp64 [G, M, N]
+ *   D[g,m,n] = C[g,m,n] + sum_{kb in g} sfa[kb][m]·sfb[kb][n]·S_kb[m,n],
+ *   S_kb[m,n] = sum_{k in kb} e4m3(A[k,m])·e4m3(B[k,n])   (exact in fp64, as for the NT GEMM).
+ * The recipe (1,1,128) gives one scale per channel (row of D for A, column of D for B) per
+ * 128-token block; a group with ks[g] == 0 gives D[g] = C[g]. */
+int dgo_k_grouped_tn(const uint8_t *a, const float *sfa, const uint8_t *b, const float *sfb,
+                     const float *c, const int *ks, int G, int M, int N, double *out) {
+    if (G <= 0 || M < 0 || N < 0) return -1;
+    size_t ldm = (size_t)pad4(M), ldn = (size_t)pad4(N);
+    int k0[4097];
+    if (G > 4096) return -1;
+    k0[0] = 0;
+    for (int g = 0; g < G; g++) {
+        if (ks[g] < 0 || ks[g] % DGO_BLK) return -2;
+        k0[g + 1] = k0[g] + ks[g];
+    }
+    double lut[256];
+    fill_lut(lut);
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int g = 0; g < G; g++) {
+        for (int m = 0; m < M; m++) {
+            for (int n = 0; n < N; n++) {
+                double acc = 0.0;
+                for (int kb = k0[g] / DGO_BLK; kb < k0[g + 1] / DGO_BLK; kb++) {
+                    double s = 0.0;
+                    for (int i = 0; i < DGO_BLK; i++) {
+                        size_t k = (size_t)kb * DGO_BLK + i;
+                        s += lut[a[k * M + m]] * lut[b[k * N + n]];
+                    }
+                    acc += (double)sfa[(size_t)kb * ldm + m] * (double)sfb[(size_t)kb * ldn + n] * s;
+                }
+                if (c) acc += (double)c[((size_t)g * M + m) * N + n];
+                out[((size_t)g * M + m) * N + n] = acc;
+            }
+        }
+    }
+    return 0;
+}
+
 int dgo_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
