@@ -50,10 +50,15 @@ def lib():
         L.dgo_m_grouped_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, P]
         L.dgo_m_grouped_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         L.dgo_cast_per_channel.argtypes = [P, I, I, P, P]
+        L.dgo_ue8m0_of_amax.restype = ctypes.c_uint8
+        L.dgo_ue8m0_of_amax.argtypes = [ctypes.c_float]
+        L.dgo_cast_per_token_ue8m0.argtypes = [P, I, I, P, P]
+        L.dgo_cast_per_block_ue8m0.argtypes = [P, I, I, I, P, P]
         L.dgo_k_grouped_tn.argtypes = [P, P, P, P, P, P, I, I, I, P]
         for f in ("dgo_cast_per_token", "dgo_cast_per_block", "dgo_transform_sf", "dgo_gemm_nt",
                   "dgo_m_grouped_contiguous", "dgo_m_grouped_masked", "dgo_num_threads",
-                  "dgo_cast_per_channel", "dgo_k_grouped_tn"):
+                  "dgo_cast_per_channel", "dgo_k_grouped_tn", "dgo_cast_per_token_ue8m0",
+                  "dgo_cast_per_block_ue8m0"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -225,3 +230,65 @@ def k_grouped_tn(a, sfa, b, sfb, ks, c=None) -> np.ndarray:
     _check(lib().dgo_k_grouped_tn(_p(a), _p(sfa), _p(b), _p(sfb), _p(c), _p(ks), G, M, N, _p(out)),
            "k_grouped_tn")
     return out
+
+
+# ------------------------------------------------------------------------------------------
+# UE8M0 (power-of-two) scales ([likun] §五: packed UE8M0 on SM100, four per 32-bit word)
+# ------------------------------------------------------------------------------------------
+
+def ue8m0_of_amax(amax: float) -> int:
+    return int(lib().dgo_ue8m0_of_amax(float(amax)))
+
+
+def cast_per_token_ue8m0(x_bf16: np.ndarray):
+    """x [M,K] bf16 bits -> (q [M,K] uint8, sfa packed uint32 [ceil(Kb/4), pad4(M)])."""
+    x = _c(x_bf16, np.uint16)
+    M, K = x.shape
+    Kb = K // 128
+    q = np.empty((M, K), np.uint8)
+    sf = np.zeros(((Kb + 3) // 4, pad4(M)), np.uint32)
+    _check(lib().dgo_cast_per_token_ue8m0(_p(x), M, K, _p(q), _p(sf)), "cast_per_token_ue8m0")
+    return q, sf
+
+
+def cast_per_block_ue8m0(x_bf16: np.ndarray):
+    """x [N,K] or [G,N,K] bf16 bits -> (q same shape, sfb packed uint32 [G?, Nb, ceil(Kb/4)])."""
+    x = _c(x_bf16, np.uint16)
+    squeeze = x.ndim == 2
+    if squeeze:
+        x = x[None]
+    G, N, K = x.shape
+    Kb = K // 128
+    q = np.empty((G, N, K), np.uint8)
+    sf = np.empty((G, (N + 127) // 128, (Kb + 3) // 4), np.uint32)
+    _check(lib().dgo_cast_per_block_ue8m0(_p(x), G, N, K, _p(q), _p(sf)), "cast_per_block_ue8m0")
+    return (q[0], sf[0]) if squeeze else (q, sf)
+
+
+def ue8m0_bytes_to_f32(b) -> np.ndarray:
+    """Scale values 2^(byte - 127) of UE8M0 bytes."""
+    return np.ldexp(np.float32(1.0), np.asarray(b, np.int32) - 127).astype(np.float32)
+
+
+def unpack_sfa_ue8m0(packed: np.ndarray, Kb: int) -> np.ndarray:
+    """[ceil(Kb/4), ld] packed words -> fp32 [Kb, ld]: K block kb is byte kb % 4 of word kb // 4."""
+    p = np.asarray(packed, np.uint32)
+    kb = np.arange(Kb)
+    bytes_ = (p[kb // 4] >> (8 * (kb % 4))[:, None].astype(np.uint32)) & 0xFF
+    return ue8m0_bytes_to_f32(bytes_)
+
+
+def unpack_sfb_ue8m0(packed: np.ndarray, Kb: int) -> np.ndarray:
+    """[G?, Nb, ceil(Kb/4)] packed words -> fp32 [G?, Nb, Kb]."""
+    p = np.asarray(packed, np.uint32)
+    kb = np.arange(Kb)
+    bytes_ = (p[..., kb // 4] >> (8 * (kb % 4)).astype(np.uint32)) & 0xFF
+    return ue8m0_bytes_to_f32(bytes_)
+
+
+def gemm_nt_ue8m0(a, sfa_packed, b, sfb_packed, c=None, rows=None) -> np.ndarray:
+    """fp64 D of the NT GEMM with UE8M0 scales: the same definition as gemm_nt, the scales
+    being the powers of two the packed bytes encode."""
+    K = np.asarray(a).shape[1]
+    Kb = K // 128
+    return gemm_nt(a, unpack_sfa_ue8m0(sfa_packed, Kb), b, unpack_sfb_ue8m0(sfb_packed, Kb), c, rows=rows)

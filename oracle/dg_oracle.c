@@ -284,6 +284,100 @@ int dgo_m_grouped_masked(const uint8_t *a, const float *sfa, const uint8_t *b, c
 }
 
 /* ---------------------------------------------------------------------------------------- */
+/* UE8M0 (power-of-two) scales ([likun] §五: on SM100 the scales are packed UE8M0, four per     */
+/* 32-bit word; §二: disable_ue8m0_cast in the fp8 GEMM's signature)                          */
+/* ---------------------------------------------------------------------------------------- */
+
+/* UE8M0 byte of a block with absolute maximum `amax`: the exponent e of the smallest power of
+ * two s = 2^e with s >= r, r = amax/448 computed as an fp32 division (the fp32 scale's own
+ * definition), stored as e + 127. amax == 0 gives s = 1 (byte 127). e is clamped to [-127, 127]. */
+uint8_t dgo_ue8m0_of_amax(float amax) {
+    if (amax == 0.0f) return 127;
+    float r = amax / 448.0f;
+    int e;
+    double f = frexp((double)r, &e);               /* r = f * 2^e, f in [0.5, 1) */
+    int ex = (f == 0.5) ? e - 1 : e;               /* r == 2^(e-1) exactly: that power itself */
+    if (ex < -127) ex = -127;
+    if (ex > 127) ex = 127;
+    return (uint8_t)(ex + 127);
+}
+
+static float ue8m0_value(uint8_t b) { return (float)ldexp(1.0, (int)b - 127); }
+
+/* Per-token cast with UE8M0 scales: as dgo_cast_per_token, with s = 2^(byte - 127) from
+ * dgo_ue8m0_of_amax (x / s is then an exact scaling before the e4m3 rounding). Scales packed
+ * four per word: sfa_packed[(kb/4) * pad4(M) + m] holds the byte of K block kb at bits
+ * 8·(kb%4); bytes of K blocks >= Kb are 127. */
+int dgo_cast_per_token_ue8m0(const uint16_t *x, int M, int K, uint8_t *q, uint32_t *sfa_packed) {
+    if (M < 0 || K <= 0 || K % DGO_BLK) return -1;
+    int Kb = K / DGO_BLK, Kq = (Kb + 3) / 4, ld = pad4(M);
+#pragma omp parallel for schedule(static)
+    for (int m = 0; m < M; m++) {
+        for (int kq = 0; kq < Kq; kq++) {
+            uint32_t word = 0;
+            for (int t = 0; t < 4; t++) {
+                int kb = 4 * kq + t;
+                uint8_t byte = 127;
+                if (kb < Kb) {
+                    const uint16_t *xs = x + (size_t)m * K + (size_t)kb * DGO_BLK;
+                    float amax = 0.0f;
+                    for (int i = 0; i < DGO_BLK; i++) {
+                        float v = fabsf(dgo_bf16_to_f32(xs[i]));
+                        if (v > amax) amax = v;
+                    }
+                    byte = dgo_ue8m0_of_amax(amax);
+                    float s = ue8m0_value(byte);
+                    for (int i = 0; i < DGO_BLK; i++)
+                        q[(size_t)m * K + (size_t)kb * DGO_BLK + i] = dgo_e4m3_encode_satrne(dgo_bf16_to_f32(xs[i]) / s);
+                }
+                word |= (uint32_t)byte << (8 * t);
+            }
+            sfa_packed[(size_t)kq * ld + m] = word;
+        }
+    }
+    return 0;
+}
+
+/* Per-block (128x128) cast with UE8M0 scales, as dgo_cast_per_block; scales packed four per
+ * word along K: sfb_packed[(g * Nb + nb) * ceil(Kb/4) + kb/4] holds block (nb, kb) at bits
+ * 8·(kb%4); bytes of K blocks >= Kb are 127. */
+int dgo_cast_per_block_ue8m0(const uint16_t *x, int batch, int N, int K, uint8_t *q, uint32_t *sfb_packed) {
+    if (batch < 0 || N < 0 || K <= 0 || K % DGO_BLK) return -1;
+    int Kb = K / DGO_BLK, Nb = (N + DGO_BLK - 1) / DGO_BLK, Kq = (Kb + 3) / 4;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int g = 0; g < batch; g++) {
+        for (int nb = 0; nb < Nb; nb++) {
+            int n_end = (nb + 1) * DGO_BLK < N ? (nb + 1) * DGO_BLK : N;
+            for (int kq = 0; kq < Kq; kq++) {
+                uint32_t word = 0;
+                for (int t = 0; t < 4; t++) {
+                    int kb = 4 * kq + t;
+                    uint8_t byte = 127;
+                    if (kb < Kb) {
+                        float amax = 0.0f;
+                        for (int n = nb * DGO_BLK; n < n_end; n++)
+                            for (int i = 0; i < DGO_BLK; i++) {
+                                float v = fabsf(dgo_bf16_to_f32(x[((size_t)g * N + n) * K + (size_t)kb * DGO_BLK + i]));
+                                if (v > amax) amax = v;
+                            }
+                        byte = dgo_ue8m0_of_amax(amax);
+                        float s = ue8m0_value(byte);
+                        for (int n = nb * DGO_BLK; n < n_end; n++)
+                            for (int i = 0; i < DGO_BLK; i++) {
+                                size_t off = ((size_t)g * N + n) * K + (size_t)kb * DGO_BLK + i;
+                                q[off] = dgo_e4m3_encode_satrne(dgo_bf16_to_f32(x[off]) / s);
+                            }
+                    }
+                    word |= (uint32_t)byte << (8 * t);
+                }
+                sfb_packed[((size_t)g * Nb + nb) * Kq + kq] = word;
+            }
+        }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------------- */
 /* K-grouped GEMM for the MoE weight gradient ([likun] §一: k_grouped_fp8_gemm_tn, "MoE 反向";  */
 /* §二: k_grouped_fp8_gemm_tn_contiguous with ks_cpu and recipe (1,1,128)).                   */
 /* ---------------------------------------------------------------------------------------- */
