@@ -50,6 +50,7 @@ def lib():
         L.dgo_m_grouped_contiguous.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, P]
         L.dgo_m_grouped_masked.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         L.dgo_cast_per_channel.argtypes = [P, I, I, P, P]
+        L.dgo_cast_per_token_scatter.argtypes = [P, P, I, I, I, P, P]
         L.dgo_ue8m0_of_amax.restype = ctypes.c_uint8
         L.dgo_ue8m0_of_amax.argtypes = [ctypes.c_float]
         L.dgo_cast_per_token_ue8m0.argtypes = [P, I, I, P, P]
@@ -58,7 +59,7 @@ def lib():
         for f in ("dgo_cast_per_token", "dgo_cast_per_block", "dgo_transform_sf", "dgo_gemm_nt",
                   "dgo_m_grouped_contiguous", "dgo_m_grouped_masked", "dgo_num_threads",
                   "dgo_cast_per_channel", "dgo_k_grouped_tn", "dgo_cast_per_token_ue8m0",
-                  "dgo_cast_per_block_ue8m0"):
+                  "dgo_cast_per_block_ue8m0", "dgo_cast_per_token_scatter"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -105,6 +106,20 @@ def cast_per_token(x_bf16: np.ndarray):
     q = np.empty((M, K), np.uint8)
     sfa = np.zeros((K // 128, pad4(M)), np.float32)
     _check(lib().dgo_cast_per_token(_p(x), M, K, _p(q), _p(sfa)), "cast_per_token")
+    return q, sfa
+
+
+def cast_per_token_scatter(x_bf16: np.ndarray, dst: np.ndarray, M_sum: int, q_init=None, sfa_init=None):
+    """Per-token cast of x [T,K] written at rows dst[t] of the contiguous layout: returns
+    (q [M_sum,K] uint8, sfa [Kb, pad4(M_sum)] fp32), starting from q_init / sfa_init (zeros when
+    None) for the rows no token maps to."""
+    x = _c(x_bf16, np.uint16)
+    T, K = x.shape
+    d = _c(dst, np.int32)
+    q = np.zeros((M_sum, K), np.uint8) if q_init is None else np.array(q_init, np.uint8, copy=True)
+    sfa = np.zeros((K // 128, pad4(M_sum)), np.float32) if sfa_init is None else np.array(sfa_init, np.float32,
+                                                                                           copy=True)
+    _check(lib().dgo_cast_per_token_scatter(_p(x), _p(d), T, K, M_sum, _p(q), _p(sfa)), "cast_per_token_scatter")
     return q, sfa
 
 

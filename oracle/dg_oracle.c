@@ -126,6 +126,41 @@ int dgo_cast_per_token(const uint16_t *x, int M, int K, uint8_t *q, float *sfa) 
     return 0;
 }
 
+/* Per-token cast straight into the M-grouped contiguous layout (the MoE dispatch of
+ * [likun] §二 m_grouped_*_contiguous, whose operand rows are the routed tokens grouped by
+ * expert): token t of x [T,K] goes to row dst[t] of q [M_sum,K] and of the MN-major sfa
+ * [Kb][pad4(M_sum)], with the per-token cast's rule; dst[t] = -1 drops the token. Rows no token
+ * maps to are not written. Every dst[t] must be < M_sum and no row may be the target of two
+ * tokens (else -2). */
+int dgo_cast_per_token_scatter(const uint16_t *x, const int32_t *dst, int T, int K, int M_sum, uint8_t *q,
+                               float *sfa) {
+    if (T < 0 || M_sum < 0 || K <= 0 || K % DGO_BLK) return -1;
+    for (int t = 0; t < T; t++)
+        if (dst[t] < -1 || dst[t] >= M_sum) return -2;
+    for (int t = 0; t < T; t++)
+        for (int u = t + 1; u < T; u++)
+            if (dst[t] >= 0 && dst[t] == dst[u]) return -2;
+    int Kb = K / DGO_BLK, ld = pad4(M_sum);
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; t++) {
+        int m = dst[t];
+        if (m < 0) continue;
+        for (int kb = 0; kb < Kb; kb++) {
+            const uint16_t *xs = x + (size_t)t * K + (size_t)kb * DGO_BLK;
+            float amax = 0.0f;
+            for (int i = 0; i < DGO_BLK; i++) {
+                float v = fabsf(dgo_bf16_to_f32(xs[i]));
+                if (v > amax) amax = v;
+            }
+            float s = scale_from_amax(amax);
+            for (int i = 0; i < DGO_BLK; i++)
+                q[(size_t)m * K + (size_t)kb * DGO_BLK + i] = dgo_e4m3_encode_satrne(dgo_bf16_to_f32(xs[i]) / s);
+            sfa[(size_t)kb * ld + m] = s;
+        }
+    }
+    return 0;
+}
+
 /* Per-block cast of weights: for every batch g, 128-row block nb and K slice kb,
  * amax over rows [nb*128, min(N, nb*128+128)) and the slice's 128 columns; then as above.
  * x: bf16 bits [batch,N,K]; q: [batch,N,K]; sfb: [batch][ceil(N/128)][Kb]. */

@@ -140,3 +140,30 @@ def test_transform_sf_matches_numpy_transpose(oracle):
     x = synth.normal_bf16(18, (6, 384))
     _, sfa = oracle.cast_per_token(x)
     assert np.array_equal(oracle.transform_sf(np.ascontiguousarray(sfa[:, :6].T)), sfa)
+
+
+def test_scatter_cast_is_the_per_token_cast_moved_to_its_rows(oracle):
+    """The cast into the contiguous layout (tokens routed to the rows of their expert's block)
+    is the per-token cast of each token, placed at its destination row; rows no token maps to
+    keep what they held, and a dropped token (-1) writes nothing."""
+    T, K, M_sum = 40, 384, 128
+    x = synth.normal_bf16(51, (T, K))
+    rng = np.random.default_rng(3)
+    dst = rng.permutation(M_sum)[:T].astype(np.int32)
+    dst[5] = -1
+    q0 = np.full((M_sum, K), 0xAB, np.uint8)
+    s0 = np.full((K // 128, M_sum), -1.0, np.float32)
+    q, sfa = oracle.cast_per_token_scatter(x, dst, M_sum, q0, s0)
+    qt, st = oracle.cast_per_token(x)
+    for t in range(T):
+        if dst[t] >= 0:
+            assert np.array_equal(q[dst[t]], qt[t])
+            assert np.array_equal(sfa[:, dst[t]], st[:, t])
+    untouched = np.setdiff1d(np.arange(M_sum), dst[dst >= 0])
+    assert np.all(q[untouched] == 0xAB) and np.all(sfa[:, untouched] == -1.0)
+
+
+def test_scatter_cast_rejects_a_row_taken_twice(oracle):
+    x = synth.normal_bf16(52, (3, 128))
+    with pytest.raises(ValueError):
+        oracle.cast_per_token_scatter(x, np.array([1, 4, 1], np.int32), 8)
