@@ -42,7 +42,8 @@
  *    For experiments and tests only (they change which kernel runs, never the result beyond
  *    the stated bound): DG_FORCE_PAIR=0|1 (CTA pairs for the tile GEMM), DG_FORCE_BN=128|256,
  *    DG_FORCE_SWAP=0|1 (few-row kernels off for M <= 128, or on for the masked layout),
- *    DG_FEW_ROW=streamk|cluster, DG_SPLITK_S=1|2|3|4|6|8|16 (cluster size). Debug only:
+ *    DG_FEW_ROW=streamk|cluster, DG_SPLITK_S=1|2|3|4|6|8|16 (cluster size), DG_ONE_ISSUER=1
+ *    (one MMA-issuing thread per CTA instead of two). Debug only:
  *    DG_TEST_SKIP_RELEASE=1|2|3 makes one kernel withhold barrier arrives or partial flags,
  *    so that a wait runs out of time (failure tests).
  */
@@ -106,6 +107,59 @@ DG_API dg_status dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, 
 DG_API dg_status dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b, const float *sfb,
                                         const void *c, void *d, int M, int N, int K, void *stream);
 
+/* Dense FP8 NT GEMM with UE8M0 (power-of-two) scales, applied by the tensor core's
+ * block-scaled MMA (likun.im §五: SM100 wants packed UE8M0 scales, four per 32-bit word; §二:
+ * disable_ue8m0_cast). D = C + A·Bᵀ with the block scaling of dg_fp8_gemm_nt, every scale
+ * being 2^(byte - 127):
+ *   a   e4m3 [M,K];   sfa uint32 [ceil(Kb/4)][pad4(M)]: byte kb%4 of word (kb/4, m) scales
+ *                     A[m, kb*128 .. kb*128+127]   (dg_cast_fp8_per_token_ue8m0 writes it)
+ *   b   e4m3 [N,K];   sfb uint32 [Nb][ceil(Kb/4)]: byte kb%4 of word (nb, kb/4) scales the
+ *                     128x128 block (nb, kb) of B   (dg_cast_fp8_per_block_ue8m0 writes it)
+ *   c   bf16 [M,N] or NULL (may alias d);   d  bf16 [M,N].
+ * Since every sfa·sfb is a power of two the hardware applies it exactly and accumulates all K
+ * blocks in TMEM (fp32). Extra precondition: N % 16 == 0. Errors as for dg_fp8_gemm_nt. */
+DG_API dg_status dg_fp8_gemm_nt_ue8m0(const void *a, const uint32_t *sfa, const void *b, const uint32_t *sfb,
+                                      const void *c, void *d, int M, int N, int K, void *stream);
+
+/* The dense GEMM in the other three storage layouts the pages name (likun.im §一,
+ * "fp8_fp4_gemm_{nt,nn,tn,tt}"; §二, "同类: _nn / _tn / _tt"). The first letter is A's
+ * storage, the second B's: A "n" = [M,K] (K contiguous), A "t" = [K,M] (M contiguous);
+ * B "t" = [N,K] (K contiguous), B "n" = [K,N] (N contiguous). The product is the NT one,
+ * D[m,n] = C[m,n] + sum_k A_log[m,k]·B_log[n,k], with the same scales:
+ *   sfa fp32 [Kb][pad4(M)] (one per row m and 128-wide K slice), sfb fp32 [Nb][Kb] (one per
+ *   128x128 block of B_log), c/d bf16 [M,N] row-major as for dg_fp8_gemm_nt.
+ *   nn: a [M,K], b [K,N];   tn: a [K,M], b [K,N];   tt: a [K,M], b [N,K].
+ * An MN-major operand reaches the tensor core through MN-major shared-memory descriptors, with
+ * no transpose pass. Extra precondition: M % 16 == 0 when A is MN-major and N % 16 == 0 when B
+ * is (16-byte rows for the tensor-map loads), else DG_ERR_INVALID_ARG. Every M takes the tile
+ * kernel (no few-row split). Errors as for dg_fp8_gemm_nt. */
+DG_API dg_status dg_fp8_gemm_nn(const void *a, const float *sfa, const void *b, const float *sfb,
+                                const void *c, void *d, int M, int N, int K, void *stream);
+DG_API dg_status dg_fp8_gemm_tn(const void *a, const float *sfa, const void *b, const float *sfb,
+                                const void *c, void *d, int M, int N, int K, void *stream);
+DG_API dg_status dg_fp8_gemm_tt(const void *a, const float *sfa, const void *b, const float *sfb,
+                                const void *c, void *d, int M, int N, int K, void *stream);
+
+/* K-grouped FP8 GEMM for the MoE weight gradient (likun.im §一, "沿 K 轴分组的
+ * k_grouped_fp8_gemm_tn（MoE 反向）"; §二, k_grouped_fp8_gemm_tn_contiguous with ks_cpu and
+ * recipe (1,1,128)). The K dimension (tokens) of both operands is cut into G consecutive groups
+ * of ks[g] tokens; group g gives D[g] = C[g] + A_gᵀ·B_g:
+ *   a   e4m3 [sum_K, M] (token-major, M contiguous: the "T" operand)
+ *   sfa fp32 [sum_K/128][pad4(M)]: one scale per channel m per 128 tokens
+ *   b   e4m3 [sum_K, N] (token-major, N contiguous: the "N" operand)
+ *   sfb fp32 [sum_K/128][pad4(N)]: one scale per channel n per 128 tokens
+ *   c   fp32 [G, M, N] or NULL (C = 0); may alias d.   d  fp32 [G, M, N], written in full.
+ *   ks         host array [G] of the group sizes, each a multiple of 128 (0 allowed: D[g] = C[g])
+ *   ks_device  the same G values in device memory (int32), read by the kernel.
+ * D[g,m,n] = C[g,m,n] + sum_{kb in g} sfa[kb][m]·sfb[kb][n]·sum_{k in kb} A[k,m]·B[k,n].
+ * Preconditions: 1 <= G <= 511, M % 16 == 0, N % 16 == 0, 16-byte aligned pointers. A device
+ * value that is not a multiple of 128 or reaches past the host's sum sets the device error word
+ * (DG_ERR_DEVICE) and its group is computed as empty. */
+DG_API dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void *a, const float *sfa, const void *b,
+                                                     const float *sfb, const float *c, float *d,
+                                                     const int *ks, const int32_t *ks_device, int G,
+                                                     int M, int N, void *stream);
+
 /* M-grouped "contiguous" FP8 NT GEMM for MoE prefill (likun.im §二,
  * m_grouped_*_gemm_nt_contiguous; zwt0204.github.io "DeepGEMM deep dive", the grouped-layout
  * constraint). The rows of A are the tokens of all G experts stacked, each expert's block
@@ -159,6 +213,46 @@ DG_API dg_status dg_cast_fp8_per_token(const void *x, void *q, float *sfa, int b
  *   x   bf16 [batch,N,K];  q e4m3 [batch,N,K];  sfb fp32 [batch][Nb][Kb]. K % 128 == 0. */
 DG_API dg_status dg_cast_fp8_per_block(const void *x, void *q, float *sfb, int batch, int N, int K,
                                 void *stream);
+
+/* The per-token cast written straight into the M-grouped contiguous layout: the MoE dispatch
+ * in front of dg_m_grouped_fp8_gemm_nt_contiguous (likun.im §二, m_grouped_*_contiguous with
+ * grouped_layout; the pages' "fused cast + grouped GEMM"). Token t of x is quantised as by
+ * dg_cast_fp8_per_token and written to row dst_rows[t] of q and sfa, in one pass, and the
+ * GEMM that follows on the stream overlaps its prologue with this kernel (programmatic
+ * dependent launch, as every kernel of the library).
+ *   x         bf16 [T,K] (tokens in any order)
+ *   dst_rows  int32 [T] on the device: the token's row in the contiguous layout, -1 to drop it;
+ *             no two tokens may share a row. A row >= M_sum sets the device error word
+ *             (DG_ERR_DEVICE) and the token is dropped.
+ *   q         e4m3 [M_sum,K];  sfa fp32 [Kb][pad4(M_sum)] (the GEMM's layouts). Rows no token
+ *             maps to (the padding of each expert's block) are not written.
+ * K % 128 == 0. */
+DG_API dg_status dg_cast_fp8_per_token_scatter(const void *x, const int32_t *dst_rows, void *q, float *sfa, int T,
+                                               int M_sum, int K, void *stream);
+
+/* Per-token and per-block FP8 casts with UE8M0 scales (likun.im §五: on SM100 the scales are
+ * packed UE8M0, four per 32-bit word; §二: disable_ue8m0_cast). The scale of a block is the
+ * smallest power of two s = 2^e >= amax/448 (the fp32 quotient), e clamped to [-127, 127]
+ * (s = 1 when amax = 0), kept as the byte e + 127; q = e4m3(x/s) as for the fp32 casts (the
+ * division by a power of two is exact). Scales are packed four K blocks per uint32 word, K
+ * block kb in bits 8·(kb%4) .. 8·(kb%4)+7; bytes of K blocks >= Kb hold 127.
+ *   per token: x bf16 [batch,M,K]; q e4m3 [batch,M,K];
+ *              sfa uint32 [batch][ceil(Kb/4)][pad4(M)] (MN-major; padding entries m >= M
+ *              are not written)
+ *   per block: x bf16 [batch,N,K]; q e4m3 [batch,N,K]; sfb uint32 [batch][Nb][ceil(Kb/4)]
+ * K % 128 == 0. */
+DG_API dg_status dg_cast_fp8_per_token_ue8m0(const void *x, void *q, uint32_t *sfa, int batch, int M, int K,
+                                             void *stream);
+DG_API dg_status dg_cast_fp8_per_block_ue8m0(const void *x, void *q, uint32_t *sfb, int batch, int N, int K,
+                                             void *stream);
+
+/* Per-channel FP8 cast along the token dimension, the recipe (1,1,128) of the K-grouped GEMM's
+ * operands (likun.im §二, k_grouped_fp8_gemm_tn_contiguous): for every 128-token block tb and
+ * channel c, amax = max_t |x[t,c]| over the block's tokens, s = amax/448 (s = 1 when amax = 0),
+ * q[t,c] = e4m3(x[t,c]/s), nearest-even, saturated to ±448 (the per-token cast's rule).
+ *   x   bf16 [T,C] token-major;  q e4m3 [T,C];  sf fp32 [T/128][pad4(C)] (padding entries are
+ *   not written). T % 128 == 0, C % 8 == 0, else DG_ERR_INVALID_ARG. */
+DG_API dg_status dg_cast_fp8_per_channel(const void *x, void *q, float *sf, int T, int C, void *stream);
 
 /* pad4(mn): the leading dimension of an MN-major scale array. */
 DG_API int dg_sf_ld(int mn);

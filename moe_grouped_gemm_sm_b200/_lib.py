@@ -54,9 +54,18 @@ def load():
             "dg_transform_sf": [P, P, I, I, I, P],
             "dg_cast_fp8_per_token": [P, P, P, I, I, I, P],
             "dg_cast_fp8_per_block": [P, P, P, I, I, I, P],
+            "dg_cast_fp8_per_channel": [P, P, P, I, I, P],
+            "dg_cast_fp8_per_token_ue8m0": [P, P, P, I, I, I, P],
+            "dg_cast_fp8_per_token_scatter": [P, P, P, P, I, I, I, P],
+            "dg_cast_fp8_per_block_ue8m0": [P, P, P, I, I, I, P],
             "dg_sf_ld": [I],
             "dg_get_device_error": [P],
             "dg_status_string": [I],
+            "dg_fp8_gemm_nt_ue8m0": [P, P, P, P, P, P, I, I, I, P],
+            "dg_fp8_gemm_nn": [P, P, P, P, P, P, I, I, I, P],
+            "dg_fp8_gemm_tn": [P, P, P, P, P, P, I, I, I, P],
+            "dg_fp8_gemm_tt": [P, P, P, P, P, P, I, I, I, P],
+            "dg_k_grouped_fp8_gemm_tn_contiguous": [P, P, P, P, P, P, P, P, I, I, I, P],
             "dg_last_kernel": [],
             "dg_allocated_bytes": [],
         }
@@ -101,6 +110,30 @@ def dg_fp8_gemm_nt_noalloc(a, sfa, b, sfb, c, d, M, N, K, stream=None):
           _stream(stream))
 
 
+def dg_fp8_gemm_nt_ue8m0(a, sfa, b, sfb, c, d, M, N, K, stream=None):
+    _call("dg_fp8_gemm_nt_ue8m0", _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(c), _ptr(d), M, N, K, _stream(stream))
+
+
+def dg_fp8_gemm_nn(a, sfa, b, sfb, c, d, M, N, K, stream=None):
+    _call("dg_fp8_gemm_nn", _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(c), _ptr(d), M, N, K, _stream(stream))
+
+
+def dg_fp8_gemm_tn(a, sfa, b, sfb, c, d, M, N, K, stream=None):
+    _call("dg_fp8_gemm_tn", _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(c), _ptr(d), M, N, K, _stream(stream))
+
+
+def dg_fp8_gemm_tt(a, sfa, b, sfb, c, d, M, N, K, stream=None):
+    _call("dg_fp8_gemm_tt", _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(c), _ptr(d), M, N, K, _stream(stream))
+
+
+def dg_k_grouped_fp8_gemm_tn_contiguous(a, sfa, b, sfb, c, d, ks, ks_device, G, M, N, stream=None):
+    """``ks`` is a sequence of G host integers (passed as a C int array), ``ks_device`` the same
+    values in an int32 device tensor."""
+    arr = (ctypes.c_int * len(ks))(*[int(k) for k in ks])
+    _call("dg_k_grouped_fp8_gemm_tn_contiguous", _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(c), _ptr(d),
+          ctypes.cast(arr, ctypes.c_void_p), _ptr(ks_device), G, M, N, _stream(stream))
+
+
 def dg_m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, c, d, grouped_layout, M_sum, N, K, G, stream=None):
     _call("dg_m_grouped_fp8_gemm_nt_contiguous", _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(c), _ptr(d),
           _ptr(grouped_layout), M_sum, N, K, G, _stream(stream))
@@ -121,6 +154,22 @@ def dg_cast_fp8_per_token(x, q, sfa, batch, M, K, stream=None):
 
 def dg_cast_fp8_per_block(x, q, sfb, batch, N, K, stream=None):
     _call("dg_cast_fp8_per_block", _ptr(x), _ptr(q), _ptr(sfb), batch, N, K, _stream(stream))
+
+
+def dg_cast_fp8_per_token_scatter(x, dst_rows, q, sfa, T, M_sum, K, stream=None):
+    _call("dg_cast_fp8_per_token_scatter", _ptr(x), _ptr(dst_rows), _ptr(q), _ptr(sfa), T, M_sum, K, _stream(stream))
+
+
+def dg_cast_fp8_per_token_ue8m0(x, q, sfa, batch, M, K, stream=None):
+    _call("dg_cast_fp8_per_token_ue8m0", _ptr(x), _ptr(q), _ptr(sfa), batch, M, K, _stream(stream))
+
+
+def dg_cast_fp8_per_block_ue8m0(x, q, sfb, batch, N, K, stream=None):
+    _call("dg_cast_fp8_per_block_ue8m0", _ptr(x), _ptr(q), _ptr(sfb), batch, N, K, _stream(stream))
+
+
+def dg_cast_fp8_per_channel(x, q, sf, T, C, stream=None):
+    _call("dg_cast_fp8_per_channel", _ptr(x), _ptr(q), _ptr(sf), T, C, _stream(stream))
 
 
 def dg_sf_ld(mn: int) -> int:

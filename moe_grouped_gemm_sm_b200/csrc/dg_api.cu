@@ -15,6 +15,7 @@
 #include "../../include/dg.h"
 #include "dg_cast.cuh"
 #include "dg_gemm.cuh"
+#include "dg_gemm_bs.cuh"
 #include "dg_gemm_splitk.cuh"
 #include "dg_gemm_swap.cuh"
 
@@ -178,6 +179,19 @@ int forced_splitk_s() {
     return v;
 }
 
+// MMA issue override for experiments (DG_ONE_ISSUER=1: one issuing thread per CTA even where
+// the stage count allows two); 0 = the kernels' own choice.
+int one_issuer() {
+    static std::atomic<int> cached{-1};
+    int v = cached.load();
+    if (v < 0) {
+        const char *s = std::getenv("DG_ONE_ISSUER");
+        v = s && std::atoi(s) ? 1 : 0;
+        cached.store(v);
+    }
+    return v;
+}
+
 // Few-row kernel by shape: the cluster split-K kernel when every tile fits one round of
 // clusters with a moderate K (its partials never leave the chip), stream-K otherwise (it splits
 // any tile count evenly over every SM, at the cost of a reduction through global memory).
@@ -234,14 +248,21 @@ bool encode(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, 
 }
 
 struct GemmMaps {
-    CUtensorMap a, b, sfa, c, d;
+    CUtensorMap a, b, sfa, c, d, sfb;
+};
+
+// Operand storage of a GEMM call: A [rows][K] or, MN-major, [K][rows]; B [G][N][K] or [G][K][N].
+struct OperandMajor {
+    bool a_mn = false, b_mn = false;
 };
 
 // Operand maps of one GEMM call. rows = rows of A/C/D per group; b_rows = rows of B one CTA
-// loads; batched = 3D maps over G groups for A, C and D (masked layout).
+// loads; batched = 3D maps over G groups for A, C and D (masked layout). MN-major operands are
+// mapped as {MN, K} boxes of 128 x 128 (one 128-byte swizzled row per K index).
 bool build_maps(GemmMaps &mp, const void *a, const float *sfa, const void *b, const void *c, void *d, int rows, int N,
-                int K, int G, int b_rows, bool batched, int slab_blocks) {
+                int K, int G, int b_rows, bool batched, int slab_blocks, OperandMajor om = OperandMajor()) {
     const uint64_t Gg = static_cast<uint64_t>(G);
+    mp.sfb = mp.sfa;   // only the K-grouped kernel reads it (build_kgrouped_maps)
     {   // sfa: fp32 [G?][Kb][pad4(rows)], box 128 x 1 (one K block's scales of a 128-row block)
         const uint64_t Kb = static_cast<uint64_t>(K / 128), ld = static_cast<uint64_t>(pad4(rows));
         const uint64_t dims[3] = {ld, Kb, Gg};
@@ -251,7 +272,13 @@ bool build_maps(GemmMaps &mp, const void *a, const float *sfa, const void *b, co
                     CU_TENSOR_MAP_SWIZZLE_NONE))
             return false;
     }
-    {   // A: e4m3 [G?][rows][K], box 128 x 128, 128-byte swizzle
+    if (om.a_mn) {   // A: e4m3 [K][rows], box 128 rows x 128 K, 128-byte swizzle
+        const uint64_t dims[2] = {static_cast<uint64_t>(rows), static_cast<uint64_t>(K)};
+        const uint64_t str[1] = {static_cast<uint64_t>(rows)};
+        const uint32_t box[2] = {128, 128};
+        if (!encode(&mp.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return false;
+    } else {   // A: e4m3 [G?][rows][K], box 128 x 128, 128-byte swizzle
         const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows), Gg};
         const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(K) * rows};
         const uint32_t box[3] = {128, 128, 1};
@@ -259,7 +286,13 @@ bool build_maps(GemmMaps &mp, const void *a, const float *sfa, const void *b, co
                     CU_TENSOR_MAP_SWIZZLE_128B))
             return false;
     }
-    {   // B: e4m3 [G][N][K], box 128 x b_rows x 1
+    if (om.b_mn) {   // B: e4m3 [G][K][N], box 128 columns x 128 K x 1 (b_rows / 128 boxes per stage)
+        const uint64_t dims[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K), Gg};
+        const uint64_t str[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(N) * K};
+        const uint32_t box[3] = {128, 128, 1};
+        if (!encode(&mp.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return false;
+    } else {   // B: e4m3 [G][N][K], box 128 x b_rows x 1
         const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), Gg};
         const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(K) * N};
         const uint32_t box[3] = {128, static_cast<uint32_t>(b_rows), 1};
@@ -307,11 +340,11 @@ struct KernelInfo {
     int max_clusters = 0;
 };
 
-template <int BN, int STAGES, int KIND, bool PAIR>
+template <int BN, int STAGES, int KIND, bool PAIR, bool A_MN = false, bool B_MN = false>
 dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p, int tiles, const DeviceInfo *di, cudaStream_t st) {
     constexpr bool PAIR_LIST = PAIR && KIND == dg::KIND_CONTIGUOUS;
-    using L = dg::GemmLayout<BN, STAGES, PAIR, PAIR_LIST>;
-    auto kern = dg::gemm_kernel<BN, STAGES, KIND, PAIR>;
+    using L = dg::GemmLayout<BN, STAGES, PAIR, PAIR_LIST, KIND == dg::KIND_KGROUPED>;
+    auto kern = dg::gemm_kernel<BN, STAGES, KIND, PAIR, A_MN, B_MN>;
     static KernelInfo info[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
@@ -336,7 +369,7 @@ dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p, int tiles, co
     const int n_units = tiles < units ? tiles : units;
     if (n_units <= 0) return DG_OK;
     cfg.gridDim = dim3(PAIR ? 2 * n_units : n_units, 1, 1);
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mp.a, mp.b, mp.sfa, mp.c, mp.d, p);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mp.a, mp.b, mp.sfa, mp.c, mp.d, mp.sfb, p);
     t_last_kernel = PAIR ? "gemm_kernel (CTA pairs)" : "gemm_kernel";
     return from_cuda(e);
 }
@@ -344,7 +377,7 @@ dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p, int tiles, co
 // Tile-shape choice. Pairs of CTAs (256-row tiles, cta_group::2) for every layout with more
 // than 128 rows per group; single CTAs (128-row tiles) otherwise. 256 columns per tile unless
 // N <= 128. Stages fill the shared-memory budget.
-template <int KIND>
+template <int KIND, bool A_MN = false, bool B_MN = false>
 dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
                    const int32_t *layout, const int32_t *masked_m, int rows, int N, int K, int G, cudaStream_t st) {
     const DeviceInfo *di = nullptr;
@@ -367,6 +400,7 @@ dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *
     p.err = di->err;
     p.timeout_ns = wait_limit_ns();
     p.test_skip_release = test_skip_release() == 1;
+    p.one_issuer = one_issuer();
     const bool batched = KIND == dg::KIND_MASKED;
     const int fbn = forced_bn();
     const int bn = fbn ? fbn : (N > 128 ? 256 : 128);
@@ -389,13 +423,74 @@ dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *
     const int b_rows = pair ? bn / 2 : bn;
     // dense and contiguous D rows in whole 64-column blocks: one TMA copy per epilogue slab
     p.cd_blocks = !batched && N % 64 == 0;
-    if (!build_maps(mp, a, sfa, b, c, d, rows, N, K, G, b_rows, batched, p.cd_blocks ? bn / 128 : 0))
+    OperandMajor om;
+    om.a_mn = A_MN;
+    om.b_mn = B_MN;
+    if (!build_maps(mp, a, sfa, b, c, d, rows, N, K, G, b_rows, batched, p.cd_blocks ? bn / 128 : 0, om))
         return DG_ERR_INVALID_ARG;
     if (pair) {
-        return launch_gemm<256, 4, KIND, true>(mp, p, tiles, di, st);
+        return launch_gemm<256, 4, KIND, true, A_MN, B_MN>(mp, p, tiles, di, st);
     }
-    if (bn == 256) return launch_gemm<256, 3, KIND, false>(mp, p, tiles, di, st);
-    return launch_gemm<128, 5, KIND, false>(mp, p, tiles, di, st);
+    if (bn == 256) return launch_gemm<256, 3, KIND, false, A_MN, B_MN>(mp, p, tiles, di, st);
+    return launch_gemm<128, 5, KIND, false, A_MN, B_MN>(mp, p, tiles, di, st);
+}
+
+// K-grouped TN GEMM (the MoE weight gradient): A [sum_K][M] and B [sum_K][N], both MN-major,
+// K split into G groups, one fp32 scale per channel per 128 tokens for both operands, fp32 D.
+dg_status run_kgrouped(const void *a, const float *sfa, const void *b, const float *sfb, const float *c, float *d,
+                       const int32_t *ks_device, int sum_k, int G, int M, int N, cudaStream_t st) {
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    dg::GemmParams p{};
+    p.M = M;
+    p.N = N;
+    p.K = sum_k;
+    p.G = G;
+    p.Kb = sum_k / 128;
+    p.Nb = (N + 127) / 128;
+    p.ld_sfa = pad4(M);
+    p.has_c = 0;
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.ks = ks_device;
+    p.d32 = d;
+    p.c32 = c;
+    p.err = di->err;
+    p.timeout_ns = wait_limit_ns();
+    p.one_issuer = one_issuer();
+    const int fbn = forced_bn();
+    const int bn = fbn ? fbn : (N > 128 ? 256 : 128);
+    const int fpair = forced_pair();
+    bool pair = fpair >= 0 ? fpair == 1 : M > 128;
+    if (bn != 256) pair = false;
+    const int m_units = (M + (pair ? 255 : 127)) / (pair ? 256 : 128);
+    p.n_blocks = (N + bn - 1) / bn;
+    const long long tiles = static_cast<long long>(G) * m_units * p.n_blocks;
+    if (tiles > (1 << 30)) return DG_ERR_INVALID_ARG;
+    p.num_tiles = static_cast<int>(tiles);
+    const int b_rows = pair ? bn / 2 : bn;
+    GemmMaps mp;
+    // With no token at all every group is empty and D = C: the kernel then loads nothing (the
+    // device offsets are clamped to p.Kb = 0), but a tensor map needs a non-empty extent.
+    const int k_ext = sum_k > 0 ? sum_k : 128;
+    {   // A [sum_K][M], B [sum_K][N] (one group of B), MN-major
+        OperandMajor om;
+        om.a_mn = om.b_mn = true;
+        if (!build_maps(mp, a, sfa, b, nullptr, d, M, N, k_ext, 1, b_rows, false, 0, om)) return DG_ERR_INVALID_ARG;
+    }
+    {   // per-column B scales fp32 [sum_K/128][pad4(N)], box bn x 1
+        const uint64_t dims[2] = {static_cast<uint64_t>(pad4(N)), static_cast<uint64_t>(k_ext / 128)};
+        const uint64_t str[1] = {static_cast<uint64_t>(pad4(N)) * 4};
+        const uint32_t box[2] = {static_cast<uint32_t>(bn), 1};
+        if (!encode(&mp.sfb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, sfb, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return DG_ERR_INVALID_ARG;
+    }
+    mp.c = mp.d = mp.sfa;   // C and D are fp32 and written directly, not through TMA
+    constexpr int KG = dg::KIND_KGROUPED;
+    if (pair) return launch_gemm<256, 4, KG, true, true, true>(mp, p, static_cast<int>(tiles), di, st);
+    if (bn == 256) return launch_gemm<256, 3, KG, false, true, true>(mp, p, static_cast<int>(tiles), di, st);
+    return launch_gemm<128, 5, KG, false, true, true>(mp, p, static_cast<int>(tiles), di, st);
 }
 
 // ---- few-row GEMMs: swapped operands, split-K over a cluster (dg_gemm_swap.cuh) ----
@@ -542,6 +637,7 @@ dg_status run_swap_with(const void *a, const float *sfa, const void *b, const fl
     p.err = di->err;
     p.timeout_ns = wait_limit_ns();
     p.test_skip_release = test_skip_streamk_flags() ? 3 : 0;
+    p.one_issuer = one_issuer();
     // the largest possible tile set: masked groups may use fewer
     const long long tiles = static_cast<long long>(batched ? G : 1) * p.m_tiles * p.n_tiles;
     SwapMaps mp;
@@ -657,6 +753,7 @@ dg_status run_splitk(const void *a, const float *sfa, const void *b, const float
     p.err = di->err;
     p.timeout_ns = wait_limit_ns();
     p.test_skip_release = test_skip_release() == 2 ? 2 : 0;
+    p.one_issuer = one_issuer();
     // tiles the cluster count is sized for: the masked layout's real count depends on masked_m,
     // estimated from expected_m
     const int m_est = batched ? (hint + tn - 1) / tn : p.m_tiles;
@@ -676,6 +773,79 @@ dg_status check_gemm_common(const void *a, const float *sfa, const void *b, cons
         (c && !aligned16(c)))
         return DG_ERR_ALIGNMENT;
     return DG_OK;
+}
+
+// UE8M0 GEMM: block-scaled MMA with the scales in TMEM (dg_gemm_bs.cuh), one CTA per 128 x 224 tile.
+dg_status run_gemm_ue8m0(const void *a, const uint32_t *sfa, const void *b, const uint32_t *sfb, const void *c,
+                         void *d, int M, int N, int K, cudaStream_t st) {
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    dg::BsParams p{};
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.Kb = K / 128;
+    p.Nb = (N + 127) / 128;
+    p.Kq = (p.Kb + 3) / 4;
+    p.ld_sfa = pad4(M);
+    p.m_blocks = (M + 127) / 128;
+    p.n_blocks = (N + dg::BS_BN - 1) / dg::BS_BN;
+    const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks;
+    if (tiles > (1 << 30)) return DG_ERR_INVALID_ARG;
+    p.num_tiles = static_cast<int>(tiles);
+    p.has_c = c != nullptr;
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.c = static_cast<const __nv_bfloat16 *>(c);
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.err = di->err;
+    p.timeout_ns = wait_limit_ns();
+    CUtensorMap tm_a, tm_b;
+    {
+        const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+        const uint64_t str[1] = {static_cast<uint64_t>(K)};
+        const uint32_t box[2] = {128, 128};
+        if (!encode(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return DG_ERR_INVALID_ARG;
+    }
+    {
+        const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
+        const uint64_t str[1] = {static_cast<uint64_t>(K)};
+        const uint32_t box[2] = {128, static_cast<uint32_t>(dg::BS_BN)};
+        if (!encode(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return DG_ERR_INVALID_ARG;
+    }
+    static std::atomic<int> ready[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
+    if (!ready[dev].load()) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!ready[dev].load()) {
+            if (cudaFuncSetAttribute(dg::gemm_bs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     dg::BsLayout::ALLOC) != cudaSuccess)
+                return DG_ERR_CUDA;
+            ready[dev].store(1);
+        }
+    }
+    const int grid = p.num_tiles < di->sm_count ? p.num_tiles : di->sm_count;
+    if (grid <= 0) return DG_OK;
+    Launch ln(dim3(static_cast<unsigned>(grid), 1, 1), dim3(dg::BS_THREADS, 1, 1), dg::BsLayout::ALLOC, st);
+    t_last_kernel = "gemm_bs_kernel (UE8M0 block-scaled MMA)";
+    return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::gemm_bs_kernel, tm_a, tm_b, p));
+}
+
+// NN / TN / TT: the dense GEMM with MN-major operands, on the tile kernel for every M.
+template <bool A_MN, bool B_MN>
+dg_status gemm_layout(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d, int M,
+                      int N, int K, void *stream) {
+    if (M < 0) return DG_ERR_INVALID_ARG;
+    dg_status s = check_gemm_common(a, sfa, b, sfb, c, d, N, K);
+    if (s != DG_OK) return s;
+    if ((A_MN && M % 16 != 0) || (B_MN && N % 16 != 0)) return DG_ERR_INVALID_ARG;   // 16-byte rows
+    if (M == 0) return DG_OK;
+    return run_gemm<dg::KIND_DENSE, A_MN, B_MN>(a, sfa, b, sfb, c, d, nullptr, nullptr, M, N, K, 1,
+                                                static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -715,6 +885,52 @@ dg_status dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b,
     return run_swap_with<dg::KIND_DENSE>(a, sfa, b, sfb, c, d, nullptr, 0, M, N, K, 1,
                                          static_cast<cudaStream_t>(stream), di, di->static_ws, di->static_flags,
                                          kStaticSlots);
+}
+
+dg_status dg_fp8_gemm_nt_ue8m0(const void *a, const uint32_t *sfa, const void *b, const uint32_t *sfb, const void *c,
+                               void *d, int M, int N, int K, void *stream) {
+    if (M < 0) return DG_ERR_INVALID_ARG;
+    dg_status s = check_gemm_common(a, reinterpret_cast<const float *>(sfa), b, reinterpret_cast<const float *>(sfb), c,
+                                    d, N, K);
+    if (s != DG_OK) return s;
+    if (N % 16 != 0) return DG_ERR_INVALID_ARG;
+    if (M == 0) return DG_OK;
+    return run_gemm_ue8m0(a, sfa, b, sfb, c, d, M, N, K, static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_fp8_gemm_nn(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
+                         int M, int N, int K, void *stream) {
+    return gemm_layout<false, true>(a, sfa, b, sfb, c, d, M, N, K, stream);
+}
+
+dg_status dg_fp8_gemm_tn(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
+                         int M, int N, int K, void *stream) {
+    return gemm_layout<true, true>(a, sfa, b, sfb, c, d, M, N, K, stream);
+}
+
+dg_status dg_fp8_gemm_tt(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
+                         int M, int N, int K, void *stream) {
+    return gemm_layout<true, false>(a, sfa, b, sfb, c, d, M, N, K, stream);
+}
+
+dg_status dg_k_grouped_fp8_gemm_tn_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
+                                              const float *c, float *d, const int *ks, const int32_t *ks_device,
+                                              int G, int M, int N, void *stream) {
+    if (!a || !sfa || !b || !sfb || !d || !ks || !ks_device || G <= 0 || G > dg::MAX_KGROUPS || M < 0 || N <= 0)
+        return DG_ERR_INVALID_ARG;
+    if (M % 16 != 0 || N % 16 != 0) return DG_ERR_INVALID_ARG;            // 16-byte rows of A and B
+    if (!aligned16(a) || !aligned16(b) || !aligned16(sfa) || !aligned16(sfb) || !aligned16(d) ||
+        (c && !aligned16(c)) || !aligned16(ks_device))
+        return DG_ERR_ALIGNMENT;
+    long long sum_k = 0;
+    for (int g = 0; g < G; ++g) {
+        if (ks[g] < 0 || ks[g] % 128 != 0) return DG_ERR_INVALID_ARG;
+        sum_k += ks[g];
+    }
+    if (sum_k > (1LL << 30)) return DG_ERR_INVALID_ARG;
+    if (M == 0) return DG_OK;
+    return run_kgrouped(a, sfa, b, sfb, c, d, ks_device, static_cast<int>(sum_k), G, M, N,
+                        static_cast<cudaStream_t>(stream));
 }
 
 dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
@@ -776,14 +992,16 @@ dg_status dg_cast_fp8_per_token(const void *x, void *q, float *sfa, int batch, i
         Launch ln(grid, dim3(256, 1, 1), 0, st);
         return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_token_kernel<32, 4>,
                                             static_cast<const __nv_bfloat16 *>(x), static_cast<uint8_t *>(q), sfa, M,
-                                            K, pad4(M)));
+                                            K, pad4(M), static_cast<const int32_t *>(nullptr), 0,
+                                            static_cast<int *>(nullptr)));
     } else {
         dim3 grid((M + 7) / 8, (Kb + 1) / 2, batch);
         if (grid.y > 65535) return DG_ERR_INVALID_ARG;
         Launch ln(grid, dim3(256, 1, 1), 0, st);
         return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_token_kernel<8, 2>,
                                             static_cast<const __nv_bfloat16 *>(x), static_cast<uint8_t *>(q), sfa, M,
-                                            K, pad4(M)));
+                                            K, pad4(M), static_cast<const int32_t *>(nullptr), 0,
+                                            static_cast<int *>(nullptr)));
     }
 }
 
@@ -797,8 +1015,80 @@ dg_status dg_cast_fp8_per_block(const void *x, void *q, float *sfb, int batch, i
     dim3 grid(K / 128, (N + 127) / 128, batch);
     if (grid.y > 65535) return DG_ERR_INVALID_ARG;
     Launch ln(grid, dim3(256, 1, 1), 0, static_cast<cudaStream_t>(stream));
-    return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_block_kernel, static_cast<const __nv_bfloat16 *>(x),
+    return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_block_kernel<false>, static_cast<const __nv_bfloat16 *>(x),
                                         static_cast<uint8_t *>(q), sfb, N, K));
+}
+
+dg_status dg_cast_fp8_per_token_scatter(const void *x, const int32_t *dst_rows, void *q, float *sfa, int T, int M_sum,
+                                       int K, void *stream) {
+    if (!x || !dst_rows || !q || !sfa || T < 0 || M_sum < 0 || K <= 0 || K % 128 != 0) return DG_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(sfa)) return DG_ERR_ALIGNMENT;
+    if (T == 0 || M_sum == 0) return DG_OK;
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    const int Kb = K / 128;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long long big_blocks = static_cast<long long>((T + 31) / 32) * ((Kb + 3) / 4);
+    if (big_blocks >= 2LL * di->sm_count) {
+        dim3 grid((T + 31) / 32, (Kb + 3) / 4, 1);
+        if (grid.y > 65535) return DG_ERR_INVALID_ARG;
+        Launch ln(grid, dim3(256, 1, 1), 0, st);
+        return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_token_kernel<32, 4, false, true>,
+                                            static_cast<const __nv_bfloat16 *>(x), static_cast<uint8_t *>(q), sfa, T, K,
+                                            pad4(M_sum), dst_rows, M_sum, di->err));
+    }
+    dim3 grid((T + 7) / 8, (Kb + 1) / 2, 1);
+    if (grid.y > 65535) return DG_ERR_INVALID_ARG;
+    Launch ln(grid, dim3(256, 1, 1), 0, st);
+    return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_token_kernel<8, 2, false, true>,
+                                        static_cast<const __nv_bfloat16 *>(x), static_cast<uint8_t *>(q), sfa, T, K,
+                                        pad4(M_sum), dst_rows, M_sum, di->err));
+}
+
+dg_status dg_cast_fp8_per_token_ue8m0(const void *x, void *q, uint32_t *sfa, int batch, int M, int K, void *stream) {
+    if (!x || !q || !sfa || batch < 0 || M < 0 || K <= 0 || K % 128 != 0 || batch > 65535) return DG_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(sfa)) return DG_ERR_ALIGNMENT;
+    if (batch == 0 || M == 0) return DG_OK;
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    const int Kq4 = (K / 128 + 3) / 4 * 4;             // the bytes of every packed word are written
+    dim3 grid((M + 31) / 32, Kq4 / 4, batch);
+    if (grid.y > 65535) return DG_ERR_INVALID_ARG;
+    Launch ln(grid, dim3(256, 1, 1), 0, static_cast<cudaStream_t>(stream));
+    return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_token_kernel<32, 4, true>,
+                                        static_cast<const __nv_bfloat16 *>(x), static_cast<uint8_t *>(q),
+                                        reinterpret_cast<float *>(sfa), M, K, pad4(M),
+                                        static_cast<const int32_t *>(nullptr), 0, static_cast<int *>(nullptr)));
+}
+
+dg_status dg_cast_fp8_per_block_ue8m0(const void *x, void *q, uint32_t *sfb, int batch, int N, int K, void *stream) {
+    if (!x || !q || !sfb || batch < 0 || N < 0 || K <= 0 || K % 128 != 0 || batch > 65535) return DG_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(sfb)) return DG_ERR_ALIGNMENT;
+    if (batch == 0 || N == 0) return DG_OK;
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    dim3 grid(K / 128, (N + 127) / 128, batch);
+    if (grid.y > 65535) return DG_ERR_INVALID_ARG;
+    Launch ln(grid, dim3(256, 1, 1), 0, static_cast<cudaStream_t>(stream));
+    return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_block_kernel<true>, static_cast<const __nv_bfloat16 *>(x),
+                                        static_cast<uint8_t *>(q), reinterpret_cast<float *>(sfb), N, K));
+}
+
+dg_status dg_cast_fp8_per_channel(const void *x, void *q, float *sf, int T, int C, void *stream) {
+    if (!x || !q || !sf || T < 0 || C < 0 || T % 128 != 0 || C % 8 != 0) return DG_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(sf)) return DG_ERR_ALIGNMENT;
+    if (T == 0 || C == 0) return DG_OK;
+    const DeviceInfo *di = nullptr;
+    dg_status s = device_info(&di);
+    if (s != DG_OK) return s;
+    dim3 grid((C + 127) / 128, T / 128, 1);
+    if (grid.y > 65535) return DG_ERR_INVALID_ARG;
+    Launch ln(grid, dim3(256, 1, 1), 0, static_cast<cudaStream_t>(stream));
+    return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::cast_per_channel_kernel, static_cast<const __nv_bfloat16 *>(x),
+                                        static_cast<uint8_t *>(q), sf, T, C, pad4(C)));
 }
 
 int dg_sf_ld(int mn) { return mn <= 0 ? 0 : pad4(mn); }

@@ -16,12 +16,25 @@
 //   warp 0      TMA producers of A (lanes 0 and 16: even and odd K blocks): A tile [128 x
 //               128 B] into a STAGES-deep ring guarded by full/empty mbarriers (for a pair, both
 //               CTAs' loads count on the leader's full barrier); they arm each stage's bytes.
-//   warp 1      TMEM allocator and (leader only) the single thread that issues tcgen05.mma
-//               kind::f8f6f4, four K=32 steps per K block, into one of 512/BN TMEM buffers, and
-//               commits the stage (empty) and the buffer (tfull) — to both CTAs of a pair.
+//               The same thread first loads the K block's A scales into a ring of their own.
+//               (A lane of a warp that waits in mbarrier.try_wait holds up the other lanes of
+//               the warp: the operand loads are kept away from any lane that waits on another
+//               ring's barriers.)
+//   warps 1, 3  (leader only) the MMA issuers, one thread each: warp 1 issues the even K
+//               blocks, warp 3 the odd ones, each tcgen05.mma kind::f8f6f4, four K=32 steps per
+//               K block, into its own TMEM buffer, and commits the stage (empty) and the buffer
+//               (tfull) — to both CTAs of a pair. A commit holds back the MMAs its thread issues
+//               after it until the committed ones are done (~800 cycles per K block with one
+//               issuer, measured); MMAs of the other thread keep the tensor pipe busy meanwhile,
+//               so with two issuers a K block costs its nominal ~540 cycles. Two issuers need an
+//               even number of stages and buffers: then every stage and buffer belongs to one
+//               issuer, which waits on its barriers phase after phase. (With an odd count a
+//               stage alternates between the issuers, and one of them could wait for a phase of
+//               a full barrier while the previous phase is still open: the parity wait would
+//               take the phase before that one, long complete, for it.) Odd stage counts keep
+//               one issuer, warp 1, which also allocates TMEM.
 //   warp 2      loads B, lanes 0 and 16 as for A (and, for contiguous pair tiles, first lists
 //               the pairs once).
-//   warp 3      loads the A-scale ring (four threads, one per K block mod 4).
 //   warps 4-11  two math warpgroups. Warp w reads TMEM lanes 32·(w%4)..+31 (its 32 rows);
 //               warpgroup j owns columns [j·BN/2, (j+1)·BN/2). Per K block: wait for the TMEM
 //               buffer, load the partial in 32-column batches (the next batch in flight while
@@ -48,13 +61,14 @@
 
 namespace dg {
 
-enum GemmKind : int { KIND_DENSE = 0, KIND_CONTIGUOUS = 1, KIND_MASKED = 2 };
+enum GemmKind : int { KIND_DENSE = 0, KIND_CONTIGUOUS = 1, KIND_MASKED = 2, KIND_KGROUPED = 3 };
 
 constexpr int BM = 128;                 // rows per CTA (one TMEM lane per row)
 constexpr int BK = 128;                 // K block = scale granularity = one 128-byte swizzle row
 constexpr int GEMM_THREADS = 384;
 constexpr int RASTER_BLOCKS = 16;       // rasterisation band height, in 128-row blocks
 constexpr int MAX_PAIR_BLOCKS = 1024;   // contiguous pair tiles: M_sum <= 1024 x 128 rows
+constexpr int MAX_KGROUPS = 511;        // K-grouped: groups whose K-block offsets fit the list area
 
 struct GemmParams {
     int M;            // rows per group of D (dense: M, contiguous: M_sum, masked: M_max)
@@ -66,16 +80,20 @@ struct GemmParams {
     int has_c;
     int cd_blocks;    // 1: C and D maps are 3D {64 columns, rows, N/64 column blocks} (one copy per slab)
     int test_skip_release;   // failure test only: warp 4 of CTA 0 skips its first TMEM release
+    int one_issuer;          // experiments: warp 1 issues every K block (no second issuer)
     const float *sfa;
     const float *sfb;
     const int32_t *grouped_layout;
     const int32_t *masked_m;
+    const int32_t *ks;       // K-grouped: tokens of each group (device), multiples of 128
     __nv_bfloat16 *d;
+    float *d32;              // K-grouped: fp32 D [G][M][N]
+    const float *c32;        // K-grouped: fp32 C [G][M][N] or NULL (may alias d32)
     int *err;
     uint64_t timeout_ns;
 };
 
-template <int BN, int STAGES, bool PAIR, bool PAIR_LIST>
+template <int BN, int STAGES, bool PAIR, bool PAIR_LIST, bool KGRP = false>
 struct GemmLayout {
     static_assert(BN % 128 == 0 && BN <= 256, "BN must be 128 or 256");
     static constexpr int HALF = BN / 2;                      // columns per math warpgroup
@@ -89,11 +107,13 @@ struct GemmLayout {
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_D = OFF_B + STAGES * B_BYTES;
     // A-scale ring: one 128-float row per K block, with full/empty barriers of its own (its
-    // loads are not on the MMA's path, so the operand ring's barriers cannot pace them).
-    static constexpr int SFS = STAGES + NBUF + 1;
+    // loads are not on the MMA's path, so the operand ring's barriers cannot pace them). The
+    // K-grouped kernel's per-column B scales (BN floats per K block) share its slots.
+    static constexpr int SFS = STAGES + NBUF + 2;
+    static constexpr int SF_SLOT = BM + (KGRP ? BN : 0);       // floats per scale slot
     static constexpr int OFF_SFA = OFF_D + 8 * SLAB_BYTES;
-    static constexpr int OFF_PAIRS = OFF_SFA + SFS * BM * 4;
-    static constexpr int PAIR_BYTES = PAIR_LIST ? MAX_PAIR_BLOCKS * 2 : 0;
+    static constexpr int OFF_PAIRS = OFF_SFA + SFS * SF_SLOT * 4;
+    static constexpr int PAIR_BYTES = PAIR_LIST ? MAX_PAIR_BLOCKS * 2 : (KGRP ? (MAX_KGROUPS + 1) * 4 : 0);
     static constexpr int OFF_BAR = OFF_PAIRS + PAIR_BYTES;
     static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 8 + 2 * SFS;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -108,6 +128,8 @@ struct TileInfo {
     int row0;     // first row (in the group's row space) of this CTA's 128-row block
     int n_blk;
     int g;
+    int kb0;      // first K block (K-grouped: the group's offset; else 0)
+    int nkb;      // K blocks of the tile (K-grouped: the group's; else Kb)
     bool valid;   // the tile exists (all CTAs of the pair agree)
     bool store;   // this CTA's rows belong to the tile's expert
 };
@@ -142,6 +164,25 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams &p, cons
     ti.valid = true;
     ti.store = true;
     ti.g = 0;
+    ti.kb0 = 0;
+    ti.nkb = p.Kb;
+    if (KIND == KIND_KGROUPED) {
+        // group-major: every group's tiles (all of them, also for an empty group, whose D is C)
+        // before the next group's, rasterised within the group; the K-block offsets of the
+        // groups sit in shared memory where the pair list would be (reinterpreted as int)
+        const int m_units = (p.M + UNIT - 1) / UNIT;
+        const int per_g = m_units * p.n_blocks;
+        const int g = t / per_g;
+        int unit, n;
+        raster(t - g * per_g, m_units, p.n_blocks, PAIR ? RASTER_BLOCKS / 2 : RASTER_BLOCKS, unit, n);
+        const int *kofs = reinterpret_cast<const int *>(pair_first);
+        ti.g = g;
+        ti.row0 = unit * UNIT + static_cast<int>(rank) * BM;
+        ti.n_blk = n;
+        ti.kb0 = kofs[g];
+        ti.nkb = kofs[g + 1] - kofs[g];
+        return ti;
+    }
     if (KIND == KIND_MASKED) {
         int rem = t;
         for (int g = 0; g < p.G; ++g) {
@@ -225,6 +266,25 @@ __device__ __forceinline__ int build_pair_list(const GemmParams &p, uint16_t *pa
     return count;
 }
 
+// K-grouped layout: one thread turns the device array of group sizes (tokens, multiples of 128)
+// into K-block offsets kofs[0..G] in shared memory. A size that is negative, not a multiple of
+// 128 or reaches past the K extent the host described sets the device error word and counts
+// as empty (its D is C).
+__device__ __forceinline__ void build_kgroup_offsets(const GemmParams &p, int *kofs) {
+    int acc = 0;
+    kofs[0] = 0;
+    for (int g = 0; g < p.G; ++g) {
+        const int k = __ldg(p.ks + g);
+        int kb = k / BK;
+        if (k < 0 || k % BK != 0 || acc + kb > p.Kb) {
+            report_error(p.err, ERR_DATA);
+            kb = 0;
+        }
+        acc += kb;
+        kofs[g + 1] = acc;
+    }
+}
+
 // tcgen05.wait::ld, then the loaded registers are read. The reads sit in the same asm statement
 // as the wait, with separate input and output operands: tied in/out operands would allow the
 // compiler to copy a register that the asynchronous load has not written yet in front of the
@@ -254,14 +314,21 @@ __device__ __forceinline__ void tmem_ld_wait_regs32(uint32_t (&r)[32]) {
     for (int i = 0; i < 32; ++i) r[i] = t[i];
 }
 
-template <int BN, int STAGES, int KIND, bool PAIR>
+// A_MN / B_MN: A stored [K, M] / B stored [K, N] (M- or N-contiguous, "T" / "N" in the
+// layout names of the pages) instead of K-contiguous; tm_a / tm_b then map those arrays and
+// the MMA reads them through MN-major descriptors. tm_sfb (K-grouped only) maps the per-column
+// B scales [Kb][pad4(N)].
+template <int BN, int STAGES, int KIND, bool PAIR, bool A_MN = false, bool B_MN = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_c,
-                const __grid_constant__ CUtensorMap tm_d, const GemmParams p) {
+                const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_sfb,
+                const GemmParams p) {
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ >= 1000)
     constexpr bool PAIR_LIST = PAIR && KIND == KIND_CONTIGUOUS;
-    using L = GemmLayout<BN, STAGES, PAIR, PAIR_LIST>;
+    constexpr bool KGRP = KIND == KIND_KGROUPED;
+    static_assert(!(A_MN || B_MN) || KIND == KIND_DENSE || KGRP, "MN-major operands: dense and K-grouped only");
+    using L = GemmLayout<BN, STAGES, PAIR, PAIR_LIST, KGRP>;
     constexpr int HALF = L::HALF;
     constexpr int NBUF = L::NBUF;
     constexpr int UNIT = PAIR ? 2 * BM : BM;
@@ -275,7 +342,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint64_t *cfull = tempty + NBUF;
     uint64_t *sfa_full = cfull + 8;
     uint64_t *sfa_empty = sfa_full + L::SFS;
-    const float *sfa_ring = reinterpret_cast<const float *>(smem + L::OFF_SFA);
+    const float *sfa_ring = reinterpret_cast<const float *>(smem + L::OFF_SFA);   // slots of SF_SLOT floats
     WaitCtx *ctx = reinterpret_cast<WaitCtx *>(smem + L::OFF_MISC);
     int *num_pairs_smem = reinterpret_cast<int *>(smem + L::OFF_MISC + sizeof(WaitCtx));
     uint16_t *pair_first = reinterpret_cast<uint16_t *>(smem + L::OFF_PAIRS);
@@ -315,6 +382,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tma_prefetch_desc(&tm_sfa);
         tma_prefetch_desc(&tm_c);
         tma_prefetch_desc(&tm_d);
+        if (KGRP) tma_prefetch_desc(&tm_sfb);
     }
     if (warp == 1) {
         if (PAIR) {
@@ -330,6 +398,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int np = build_pair_list(p, pair_first, lane);
         if (lane == 0) *num_pairs_smem = np;
     }
+    if (KGRP && warp == 2 && lane == 0) build_kgroup_offsets(p, reinterpret_cast<int *>(pair_first));
     tc_fence_before();
     if (PAIR)
         cluster_sync();
@@ -355,14 +424,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         reg_dealloc<56>();
         // TMA producers. One thread's bulk copies are served one after another (a fixed cost
         // per copy, whatever its size), so A and B each get two threads (lanes 0 and 16 of warps
-        // 0 and 2: even and odd K blocks) and the small A-scale copies four (lanes 0, 8, 16, 24
-        // of warp 3: K block mod 4); the A thread of a K block arms its stage. All wait on the same "empty" barriers of the ring; none can run
-        // more than STAGES K blocks ahead of the others, since a stage is only freed once all
-        // its loads have landed and the MMA has consumed it.
-        const int stream = warp == 0 || warp == 2 ? ((lane & 15) == 0 ? warp >> 1 : -1) : (warp == 3 && (lane & 7) == 0 ? 2 : -1);
-        // A/B (weights/activations): K block parity = lane / 16; A scales: K block mod 4 = lane / 8
-        const uint32_t parity = static_cast<uint32_t>(stream == 2 ? lane >> 3 : lane >> 4);
-        const uint32_t nlanes = stream == 2 ? 4u : 2u;
+        // 0 and 2: even and odd K blocks); the A thread of a K block also loads its A scales
+        // (into a slot of their ring, whose release by the math warps is at most STAGES + NBUF
+        // K blocks behind, less than the ring's SFS slots) and arms its stage. All wait on the
+        // same "empty" barriers of the operand ring; none can run more than STAGES K blocks
+        // ahead of the others, since a stage is only freed once all its loads have landed and
+        // the MMA has consumed it.
+        const int stream = (warp == 0 || warp == 2) && (lane & 15) == 0 ? warp >> 1 : -1;
+        const uint32_t parity = static_cast<uint32_t>(lane >> 4);
+        const uint32_t nlanes = 2u;
         if (stream >= 0) {
             uint32_t it = 0;
             for (int t = cid; t < num_tiles && !*abort_flag; t += ncid) {
@@ -372,20 +442,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     continue;
                 }
                 const int brow = ti.n_blk * BN + static_cast<int>(rank) * L::B_ROWS;
-                for (int kb = 0; kb < p.Kb; ++kb, ++it) {
+                const int bz = KGRP ? 0 : ti.g;                    // K-grouped B: one [sum_K, N] array
+                const int nkb = KGRP ? ti.nkb : p.Kb;
+                for (int kbl = 0; kbl < nkb; ++kbl, ++it) {
                     if (it % nlanes != parity) continue;
+                    const int kb = KGRP ? ti.kb0 + kbl : kbl;      // K block in the operands' K space
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (stream == 2) {
+                    if (stream == 0) {
                         const int j = it % L::SFS;
                         if (!mbar_wait(&sfa_empty[j], ((it / L::SFS) & 1) ^ 1, ctx)) break;
-                        float *sf = reinterpret_cast<float *>(smem + L::OFF_SFA) + j * BM;
-                        mbar_arrive_expect_tx(&sfa_full[j], BM * 4);
+                        float *sf = reinterpret_cast<float *>(smem + L::OFF_SFA) + j * L::SF_SLOT;
+                        mbar_arrive_expect_tx(&sfa_full[j], L::SF_SLOT * 4);
                         if (KIND == KIND_MASKED)
                             tma_load_3d(&tm_sfa, &sfa_full[j], sf, ti.row0, kb, ti.g);
                         else
                             tma_load_2d(&tm_sfa, &sfa_full[j], sf, ti.row0, kb);
-                        continue;
+                        if (KGRP) tma_load_2d(&tm_sfb, &sfa_full[j], sf + BM, ti.n_blk * BN, kb);
                     }
                     if (!mbar_wait(&empty[s], ph ^ 1, ctx)) break;
                     uint8_t *sa = smem + L::OFF_A + s * L::A_BYTES;
@@ -394,48 +467,75 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);   // the leader's barrier
                         if (stream == 0) {
                             if (leader) mbar_arrive_expect_tx(&full[s], L::STAGE_TX);
-                            if (KIND == KIND_MASKED)
+                            if (A_MN)
+                                tma_load_2d_pair(&tm_a, fb, sa, ti.row0, kb * BK);
+                            else if (KIND == KIND_MASKED)
                                 tma_load_3d_pair(&tm_a, fb, sa, kb * BK, ti.row0, ti.g);
                             else
                                 tma_load_2d_pair(&tm_a, fb, sa, kb * BK, ti.row0);
+                        } else if (B_MN) {
+#pragma unroll
+                            for (int i = 0; i < L::B_ROWS / 128; ++i)
+                                tma_load_3d_pair(&tm_b, fb, sb + i * 128 * BK, brow + 128 * i, kb * BK, bz);
                         } else {
-                            tma_load_3d_pair(&tm_b, fb, sb, kb * BK, brow, ti.g);
+                            tma_load_3d_pair(&tm_b, fb, sb, kb * BK, brow, bz);
                         }
                     } else {
                         if (stream == 0) {
                             mbar_arrive_expect_tx(&full[s], L::STAGE_TX);
-                            if (KIND == KIND_MASKED)
+                            if (A_MN)
+                                tma_load_2d(&tm_a, &full[s], sa, ti.row0, kb * BK);
+                            else if (KIND == KIND_MASKED)
                                 tma_load_3d(&tm_a, &full[s], sa, kb * BK, ti.row0, ti.g);
                             else
                                 tma_load_2d(&tm_a, &full[s], sa, kb * BK, ti.row0);
+                        } else if (B_MN) {
+#pragma unroll
+                            for (int i = 0; i < L::B_ROWS / 128; ++i)
+                                tma_load_3d(&tm_b, &full[s], sb + i * 128 * BK, brow + 128 * i, kb * BK, bz);
                         } else {
-                            tma_load_3d(&tm_b, &full[s], sb, kb * BK, brow, ti.g);
+                            tma_load_3d(&tm_b, &full[s], sb, kb * BK, brow, bz);
                         }
                     }
                 }
             }
-        } else if (warp == 1 && lane == 0 && leader) {
-            // ---------------- MMA issuer (the leader CTA of a pair) ----------------
-            constexpr uint32_t IDESC = idesc_f8_e4m3_f32<UNIT, BN>();
+        } else if ((warp == 1 || (warp == 3 && STAGES % 2 == 0 && NBUF % 2 == 0 && !p.one_issuer)) && lane == 0 &&
+                   leader) {
+            // ---------------- MMA issuers (the leader CTA of a pair) ----------------
+            // warp 1: K blocks with an even running index, warp 3: odd ones; both stage and
+            // buffer counts even, so each issuer owns its stages and TMEM buffers
+            constexpr bool TWO_OK = STAGES % 2 == 0 && NBUF % 2 == 0;
+            const bool two = TWO_OK && !p.one_issuer;
+            const uint32_t mine = warp == 1 ? 0u : 1u;
+            constexpr uint32_t IDESC = idesc_f8_e4m3_f32<UNIT, BN, A_MN, B_MN>();
+            // a K step of 32: 32 bytes along a K-major row (+2 in the 16-byte granular start
+            // address), or 32 rows of 128 bytes of an MN-major tile (+256)
+            constexpr uint64_t A_STEP = A_MN ? 256 : 2, B_STEP = B_MN ? 256 : 2;
             uint32_t it = 0;
             for (int t = cid; t < num_tiles && !*abort_flag; t += ncid) {
                 const TileInfo ti = decode_tile<KIND, PAIR>(t, p, pair_first, num_pairs, rank);
                 if (!ti.valid) continue;
-                for (int kb = 0; kb < p.Kb; ++kb, ++it) {
+                const int nkb = KGRP ? ti.nkb : p.Kb;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    if (two && (it & 1u) != mine) continue;
                     const int s = it % STAGES;
                     const int b = it % NBUF;
                     if (!mbar_wait(&full[s], (it / STAGES) & 1, ctx)) break;
                     if (!mbar_wait(&tempty[b], ((it / NBUF) & 1) ^ 1, ctx)) break;
                     tc_fence_after();
-                    const uint64_t ad = sdesc_k_sw128(smem_u32(smem + L::OFF_A + s * L::A_BYTES));
-                    const uint64_t bd = sdesc_k_sw128(smem_u32(smem + L::OFF_B + s * L::B_BYTES));
+                    const uint32_t a_addr = smem_u32(smem + L::OFF_A + s * L::A_BYTES);
+                    const uint32_t b_addr = smem_u32(smem + L::OFF_B + s * L::B_BYTES);
+                    // MN-major: 128-element atoms 128 rows x 128 bytes apart (the second B atom
+                    // of a 256-column single-CTA tile)
+                    const uint64_t ad = A_MN ? sdesc_mn_sw128(a_addr, 128 * BK) : sdesc_k_sw128(a_addr);
+                    const uint64_t bd = B_MN ? sdesc_mn_sw128(b_addr, 128 * BK) : sdesc_k_sw128(b_addr);
                     const uint32_t dt = tmem_base + static_cast<uint32_t>(b * BN);
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k) {
                         if (PAIR)
-                            umma_f8_pair(dt, ad + 2 * k, bd + 2 * k, IDESC, k > 0 ? 1u : 0u);
+                            umma_f8_pair(dt, ad + A_STEP * k, bd + B_STEP * k, IDESC, k > 0 ? 1u : 0u);
                         else
-                            umma_f8(dt, ad + 2 * k, bd + 2 * k, IDESC, k > 0 ? 1u : 0u);
+                            umma_f8(dt, ad + A_STEP * k, bd + B_STEP * k, IDESC, k > 0 ? 1u : 0u);
                     }
                     if (PAIR) {
                         umma_commit_pair(&empty[s], 0x3);
@@ -465,7 +565,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const int row = srow0 + lane;                        // this thread's row
             const int nblk = min(col0 / 128, p.Nb - 1);
             const float *sfb_row = p.sfb + (static_cast<size_t>(ti.g) * p.Nb + nblk) * p.Kb;
-            const bool do_c = p.has_c && ti.store;
+            const bool do_c = !KGRP && p.has_c && ti.store;
             if (do_c && lane == 0) {
                 bulk_wait_group_read0();                         // the slab's last store has read it
                 fence_proxy_async_smem();
@@ -488,32 +588,37 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             // sfb of this warp's n-block, 32 K blocks per window (one value per lane, broadcast by
             // shuffle); sfa of this thread's row from the TMA-filled ring. No global load is left
             // in flight across the loop's release-arrives except a window refill every 32 blocks.
-            float sb_win = lane < p.Kb ? __ldg(sfb_row + lane) : 0.f;
-            float sb_nxt = 32 + lane < p.Kb ? __ldg(sfb_row + 32 + lane) : 0.f;
-            for (int kb = 0; kb < p.Kb; ++kb, ++it) {
+            // (K-grouped: one B scale per column, from the same ring slot as sfa)
+            float sb_win = !KGRP && lane < p.Kb ? __ldg(sfb_row + lane) : 0.f;
+            float sb_nxt = !KGRP && 32 + lane < p.Kb ? __ldg(sfb_row + 32 + lane) : 0.f;
+            const int nkb = KGRP ? ti.nkb : p.Kb;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int b = it % NBUF;
                 const uint32_t phb = (it / NBUF) & 1;
-                if ((kb & 31) == 0 && kb > 0) {
+                if (!KGRP && (kb & 31) == 0 && kb > 0) {
                     sb_win = sb_nxt;
                     sb_nxt = kb + 32 + lane < p.Kb ? __ldg(sfb_row + kb + 32 + lane) : 0.f;
                 }
-                const float sb = __shfl_sync(0xFFFFFFFFu, sb_win, kb & 31);
+                const float sb = KGRP ? 1.f : __shfl_sync(0xFFFFFFFFu, sb_win, kb & 31);
                 const int j = it % L::SFS;
                 // every lane waits; the outcome is made warp-uniform before any .sync.aligned op
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], phb, ctx));
                 if (!ok) break;
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sfa_full[j], (it / L::SFS) & 1, ctx));
                 if (!ok) break;
-                const float sa = sfa_ring[j * BM + q * 32 + lane];
+                const float sa = sfa_ring[j * L::SF_SLOT + q * 32 + lane];
                 tc_fence_after();
                 const float scale = sa * sb;
-                // the slot is read: the generic-proxy read is ordered before the producer's next
-                // TMA write into the slot (async proxy) by a proxy fence, which release/acquire
-                // through the mbarrier alone does not give
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_relaxed(&sfa_empty[j]);
+                if (!KGRP) {
+                    // the slot is read: the generic-proxy read is ordered before the producer's
+                    // next TMA write into the slot (async proxy) by a proxy fence, which
+                    // release/acquire through the mbarrier alone does not give
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_relaxed(&sfa_empty[j]);
+                }
                 const float2 scale2 = make_float2(scale, scale);
+                const float *sbc = sfa_ring + j * L::SF_SLOT + BM + wg * HALF;   // K-grouped column scales
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                        static_cast<uint32_t>(b * BN + wg * HALF);
                 // 32-column batches, double-buffered in registers: the TMEM load of batch c+1 is
@@ -527,13 +632,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     if (c + 1 < HALF / 32) tmem_ld32(taddr + (c + 1) * 32, r[(c + 1) & 1]);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {   // packed fp32x2 FMA: half the issue slots
+                        float2 s2 = scale2;
+                        if (KGRP) {                   // sa · sfb[column], sfb broadcast from shared memory
+                            const float2 sb2 = *reinterpret_cast<const float2 *>(sbc + c * 32 + 2 * i);
+                            s2 = __fmul2_rn(scale2, sb2);
+                        }
                         const float2 a2 = __ffma2_rn(
-                            make_float2(__uint_as_float(r[c & 1][2 * i]), __uint_as_float(r[c & 1][2 * i + 1])), scale2,
+                            make_float2(__uint_as_float(r[c & 1][2 * i]), __uint_as_float(r[c & 1][2 * i + 1])), s2,
                             make_float2(acc[c * 32 + 2 * i], acc[c * 32 + 2 * i + 1]));
                         acc[c * 32 + 2 * i] = a2.x;
                         acc[c * 32 + 2 * i + 1] = a2.y;
                     }
                     if (c + 1 < HALF / 32) tmem_ld_wait_regs32(r[(c + 1) & 1]);
+                }
+                if (KGRP) {                            // the column scales are read too
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_relaxed(&sfa_empty[j]);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -548,6 +663,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             }
             if (!ok) break;
             if (!ti.store) continue;
+            if (KGRP) {
+                // fp32 D (a weight gradient): each thread stores its row's HALF columns, 16 bytes
+                // at a time, after adding C (read the same way; N % 16 == 0, so a 4-column
+                // vector is all in or all out)
+                if (row < p.M) {
+                    const size_t rbase = (static_cast<size_t>(ti.g) * p.M + row) * p.N;
+#pragma unroll
+                    for (int c4 = 0; c4 < HALF / 4; ++c4) {
+                        const int col = col0 + c4 * 4;
+                        if (col < p.N) {
+                            float4 v = make_float4(acc[4 * c4], acc[4 * c4 + 1], acc[4 * c4 + 2], acc[4 * c4 + 3]);
+                            if (p.c32) {
+                                const float4 cv = *reinterpret_cast<const float4 *>(p.c32 + rbase + col);
+                                v.x += cv.x;
+                                v.y += cv.y;
+                                v.z += cv.z;
+                                v.w += cv.w;
+                            }
+                            *reinterpret_cast<float4 *>(p.d32 + rbase + col) = v;
+                        }
+                    }
+                }
+                continue;
+            }
             if (do_c) {
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&cfull[mw], ctile & 1, ctx));
                 if (!ok) break;

@@ -17,16 +17,19 @@
 //     reducer's mbarrier), so CTA j receives its rows [8·floor(16j/S), 8·floor(16(j+1)/S)) of
 //     all S partials, sums them in rank order (deterministic), adds C and writes D. No global
 //     workspace, no flags: the partials stay on chip;
-//   * one tcgen05.commit per K block. A commit drains the tensor pipe: four M=128 MMAs and their
-//     commit take ~830 cycles whatever N is, against ~355 per K block for N = 64 with one commit
-//     per four K blocks. But each SM streams a K block's 24-32 KB in ~1000 cycles here, so the
-//     MMA has the slack, and grouping commits (KG > 1) only delays the promotion (measured
-//     slower).
+//   * one tcgen05.commit per K block, from two issuing threads when the stage count is even.
+//     A commit holds back the MMAs its thread issues after it until the committed ones are
+//     done: four M=128 MMAs and their commit take ~800 cycles whatever N is when one thread
+//     issues everything. With the even and the odd K blocks on two threads, each owning its
+//     stages and TMEM buffers, the other thread's MMAs keep the tensor pipe busy meanwhile.
+//     (An odd stage count keeps one issuer: a stage shared by both could see one issuer wait
+//     on a full barrier a phase early.)
 //
-// CTA layout: warps 0, 2, 3 TMA producers (weights and activations on two threads each, the A
-// scales on four), warp 1 TMEM allocator + single-thread tcgen05.mma issuer (kind::f8f6f4,
-// M = 128, N = TN), warps 4-11 two math warpgroups (thread = weight row, registers = its
-// warpgroup's TN/2 token columns), which also push, reduce and store.
+// CTA layout: warps 0 and 2 TMA producers (weights and activations on two threads each, the A
+// scales on four), warps 1 and 3 the tcgen05.mma issuers (kind::f8f6f4, M = 128, N = TN, even
+// and odd K blocks; warp 1 also allocates TMEM), warps 4-11 two math warpgroups (thread =
+// weight row, registers = its warpgroup's TN/2 token columns), which also push, reduce and
+// store.
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -196,9 +199,10 @@ __global__ void __launch_bounds__(SplitLayout<TN, STAGES>::THREADS, 1)
 
     if (warp < 4) {
         // TMA producers: lanes 0 and 16 of warps 0 (weights) and 2 (activations), even and odd
-        // K blocks; lanes 0, 8, 16, 24 of warp 3 (A scales), K block mod 4.
-        const int stream = warp == 0 || warp == 2 ? ((lane & 15) == 0 ? warp >> 1 : -1) : (warp == 3 && (lane & 7) == 0 ? 2 : -1);
-        const uint32_t parity = static_cast<uint32_t>(stream == 2 ? lane >> 3 : lane >> 4);
+        // K blocks; lanes 8 and 24 of warps 0 and 2 (A scales), K block mod 4.
+        const bool is_producer = (warp == 0 || warp == 2) && (lane & 7) == 0;
+        const int stream = !is_producer ? -1 : ((lane & 15) == 0 ? warp >> 1 : 2);
+        const uint32_t parity = static_cast<uint32_t>(stream == 2 ? 2 * (warp >> 1) + (lane >> 4) : lane >> 4);
         const uint32_t nlanes = stream == 2 ? 4u : 2u;
         if (stream >= 0) {
             const uint64_t pol = stream == 0 ? l2_policy_evict_first() : l2_policy_evict_last();
@@ -230,14 +234,22 @@ __global__ void __launch_bounds__(SplitLayout<TN, STAGES>::THREADS, 1)
                     }
                 }
             }
-        } else if (warp == 1 && lane == 0) {
-            // ---------------- MMA issuer: a commit per KG K blocks and at each tile's end ----------------
+        } else if ((warp == 1 || (warp == 3 && STAGES % 2 == 0 && NBUF % 2 == 0 && !p.one_issuer)) && lane == 0) {
+            // ---------------- MMA issuers: warp 1 even K blocks, warp 3 odd ones ----------------
+            // (a commit holds back only the MMAs its own thread issues after it, so the other
+            // issuer keeps the tensor pipe busy while one waits; each has its own TMEM buffers)
+            // two issuers need even stage and buffer counts (each issuer then owns its stages
+            // and buffers and waits on their barriers phase after phase); odd counts keep one
+            static_assert(KG == 1, "one commit per K block");
+            const bool two = STAGES % 2 == 0 && NBUF % 2 == 0 && !p.one_issuer;
+            const uint32_t mine = warp == 1 ? 0u : 1u;
             constexpr uint32_t IDESC = idesc_f8_e4m3_f32<128, TN>();
             uint32_t it = 0;
             bool ok = true;
             for (int tile = cid; tile < tiles.count && ok; tile += nclusters) {
                 int pending = 0;
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    if (two && (it & 1u) != mine) continue;
                     const int s = it % STAGES;
                     const int b = it % NBUF;
                     ok = mbar_wait(&full[s], (it / STAGES) & 1, ctx) && mbar_wait(&tempty[b], ((it / NBUF) & 1) ^ 1, ctx);

@@ -26,10 +26,10 @@
 //     matches, no flag needs clearing, and CUDA-graph replays stay valid;
 //   * a deep TMA ring (5-8 stages of the 16 KB weight tile) keeps enough bytes in flight.
 //
-// CTA layout: warps 0, 2, 3 TMA producers (weights and activations on two threads each, the A
-// scales on four), warp 1 TMEM allocator + single-thread tcgen05.mma issuer (kind::f8f6f4,
-// M = 128, N = TN), warps 4-11 two math warpgroups (thread = weight row, registers = its
-// warpgroup's TN/2 token columns).
+// CTA layout: warps 0 and 2 TMA producers (weights and activations on two threads each, the A
+// scales on four), warps 1 and 3 the tcgen05.mma issuers (kind::f8f6f4, M = 128, N = TN), one
+// thread each for the even and the odd K blocks (warp 1 also allocates TMEM), warps 4-11 two
+// math warpgroups (thread = weight row, registers = its warpgroup's TN/2 token columns).
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -59,6 +59,7 @@ struct SwapParams {
     // failure tests only: 2 = the cluster kernel's CTA 0, warp 4 withholds its first push
     // arrive; 3 = the stream-K kernel's odd-numbered CTAs withhold their partial flags
     int test_skip_release;
+    int one_issuer;   // experiments: warp 1 issues every K block (no second issuer)
 };
 
 // Ticket of a stream-K launch: one past the epoch word, never 0 (flags start out zero).
@@ -241,9 +242,11 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
         // odd K blocks) and the small A-scale copies four (lanes 0, 8, 16, 24 of warp 3, K block
         // mod 4). The weight thread of a K block arms its stage. All wait on the ring's "empty"
         // barriers.
-        const int stream = warp == 0 || warp == 2 ? ((lane & 15) == 0 ? warp >> 1 : -1) : (warp == 3 && (lane & 7) == 0 ? 2 : -1);
-        // A/B (weights/activations): K block parity = lane / 16; A scales: K block mod 4 = lane / 8
-        const uint32_t parity = static_cast<uint32_t>(stream == 2 ? lane >> 3 : lane >> 4);
+        const bool is_producer = (warp == 0 || warp == 2) && (lane & 7) == 0;
+        const int stream = !is_producer ? -1 : ((lane & 15) == 0 ? warp >> 1 : 2);
+        // weights/activations: K block parity = lane / 16; A scales (lanes 8 and 24 of warps 0
+        // and 2): K block mod 4 = 2·(warp / 2) + lane / 16
+        const uint32_t parity = static_cast<uint32_t>(stream == 2 ? 2 * (warp >> 1) + (lane >> 4) : lane >> 4);
         const uint32_t nlanes = stream == 2 ? 4u : 2u;
         if (stream >= 0) {
             // the weights are read once: evict them first; activations and A scales are read
@@ -279,8 +282,15 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
                     }
                 }
             }
-        } else if (warp == 1 && lane == 0) {
-            // ---------------- MMA issuer ----------------
+        } else if ((warp == 1 || (warp == 3 && STAGES % 2 == 0 && NBUF % 2 == 0 && !p.one_issuer)) && lane == 0) {
+            // ---------------- MMA issuers: warp 1 even K blocks, warp 3 odd ones ----------------
+            // (a commit holds back only the MMAs its own thread issues after it, so the other
+            // issuer keeps the tensor pipe busy while one waits; each has its own TMEM buffers)
+            // two issuers need even stage and buffer counts (each issuer then owns its stages
+            // and buffers and waits on their barriers phase after phase); odd counts keep one
+            static_assert(L::KG == 1, "one commit per K block");
+            const bool two = STAGES % 2 == 0 && NBUF % 2 == 0 && !p.one_issuer;
+            const uint32_t mine = warp == 1 ? 0u : 1u;
             constexpr uint32_t IDESC = idesc_f8_e4m3_f32<128, TN>();
             // one commit per K block (KG = 1): grouping commits, which saves tensor-pipe drains,
             // measured slower here, where the run is bandwidth-bound and the tile tails matter
@@ -292,6 +302,7 @@ __global__ void __launch_bounds__(SwapLayout<TN, STAGES>::THREADS, 1)
                 u += kbe - kbs;
                 int pending = 0;
                 for (int kb = kbs; kb < kbe; ++kb, ++it) {
+                    if (two && (it & 1u) != mine) continue;
                     const int s = it % STAGES;
                     const int b = it % NBUF;
                     ok = mbar_wait(&full[s], (it / STAGES) & 1, ctx) && mbar_wait(&tempty[b], ((it / NBUF) & 1) ^ 1, ctx);

@@ -275,14 +275,30 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile written by TMA with 128-byte
+// swizzle: each K row holds 128 consecutive M (or N) elements in 128 bytes, 8-row groups 1024
+// bytes apart (stride byte offset), and further 128-element MN atoms `lbo` bytes apart
+// (leading byte offset); version 1, layout type 2 = SWIZZLE_128B. A K step of 32 rows adds
+// 4096 bytes (256 in the 16-byte granular start address).
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
 // Instruction descriptor of tcgen05.mma kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B E4M3
-// (format 0 at bits 7-9 and 10-12), both K-major (bits 15, 16 = 0), N>>3 at bits 17-22,
-// M>>4 at bits 24-28.
-template <int M_, int N_>
+// (format 0 at bits 7-9 and 10-12), A and B K-major (bits 15, 16 = 0) or MN-major (1), N>>3
+// at bits 17-22, M>>4 at bits 24-28.
+template <int M_, int N_, bool A_MN = false, bool B_MN = false>
 __host__ __device__ constexpr uint32_t idesc_f8_e4m3_f32() {
     static_assert(M_ == 64 || M_ == 128 || M_ == 256, "MMA M");
     static_assert(N_ % 8 == 0 && N_ >= 8 && N_ <= 256, "MMA N");
-    return (1u << 4) | (static_cast<uint32_t>(N_ >> 3) << 17) | (static_cast<uint32_t>(M_ >> 4) << 24);
+    return (1u << 4) | (static_cast<uint32_t>(A_MN) << 15) | (static_cast<uint32_t>(B_MN) << 16) |
+           (static_cast<uint32_t>(N_ >> 3) << 17) | (static_cast<uint32_t>(M_ >> 4) << 24);
 }
 
 // D[tmem] (+)= A[smem] · B[smem]ᵀ, one CTA, issued by a single thread.

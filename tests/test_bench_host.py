@@ -35,8 +35,10 @@ def test_every_page_configuration_is_measured():
     """The headline (prefill) plus the workloads object cover every configuration of the pages:
     the 64x2112x7168 C = 0 decode shape, decode M = 64 and 128 cold and warm, contiguous, masked."""
     keys = {k for k, _, _ in bench.SUB_WORKLOADS}
-    assert keys == {"config1", "decode64_cold", "decode64_warm", "decode128_cold", "decode128_warm",
-                    "contiguous", "masked"}
+    assert {"config1", "decode64_cold", "decode64_warm", "decode128_cold", "decode128_warm",
+            "contiguous", "masked"} <= keys
+    # and the rows beyond the page configurations: the other layouts and the K-grouped GEMM
+    assert {"layouts", "k_grouped"} <= keys
     c1 = bench.WORKLOADS["config1"]
     assert c1["M"] == 64 and c1["shapes"] == [(2112, 7168)] and not c1["with_c"]
     for name in ("decode64", "decode128"):
@@ -63,3 +65,16 @@ def test_stored_traffic_is_dropped_when_the_kernels_change(tmp_path, monkeypatch
     assert bench.stored_traffic("prefill") == 123.0
     assert bench.stored_traffic("decode64") is None
     assert bench.stored_traffic("masked") is None
+
+
+def test_k_grouped_problem_sizes_and_bytes():
+    """The K-grouped workload: G = 8 groups of U{2048..6144} tokens padded to 128, gradient
+    shapes (M,N) from the expert weights; bytes = both e4m3 operands, their per-channel scales
+    and the fp32 D."""
+    probs = bench.make_problems(dict(bench.WORKLOADS["k_grouped"], shapes=[(256, 128)]))
+    (p,) = probs
+    assert len(p["ks"]) == 8 and all(k % 128 == 0 and 2048 <= k <= 6144 + 127 for k in p["ks"])
+    T = sum(p["ks"])
+    assert p["K"] == T and p["x"].shape == (T, 256) and p["w"].shape == (T, 128)
+    assert p["flops"] == 2.0 * 256 * 128 * T
+    assert bench.algorithmic_bytes(p) == T * 256 + T * 128 + 4 * (T // 128) * (256 + 128) + 4 * 8 * 256 * 128
