@@ -38,6 +38,7 @@ of the same workload; under torchrun only rank 0 runs it.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -62,10 +63,21 @@ WORKLOADS = {
                       desc="dense FP8 NT GEMM, M=128 decode, six (N,K) shapes, C bf16"),
     "contiguous": dict(kind="contiguous", G=8, shapes=GROUPED_SHAPES, with_c=False,
                        desc="M-grouped contiguous FP8 GEMM, G=8, m_g ~ U{2048..6144} padded to 128, "
-                            "(N,K) in {(4096,7168),(7168,2048)}"),
+                            "(N,K) in {(4096,7168),(7168,2048)}; the step's cast takes the routed tokens "
+                            "(shuffled) straight into the grouped layout"),
     "masked": dict(kind="masked", G=16, M_max=256, expected_m=192, shapes=GROUPED_SHAPES, with_c=False,
                    desc="M-grouped masked FP8 GEMM, G=16, M_max=256, masked_m ~ U{64..256}, expected_m=192, "
                         "(N,K) in {(4096,7168),(7168,2048)}"),
+    "prefill_ue8m0": dict(kind="dense", M=4096, shapes=PREFILL_SHAPES, with_c=True, ue8m0=True,
+                          desc="dense FP8 NT GEMM with UE8M0 (power-of-two) scales and the block-scaled MMA, M=4096, "
+                               "the six prefill (N,K) shapes, C bf16"),
+    "layouts": dict(kind="layout", M=4096, shapes=[(4096, 7168)], layouts=("nn", "tn", "tt"), with_c=True,
+                    desc="dense FP8 GEMM, M=4096, N=4096, K=7168, C bf16, in the NN, TN and TT storage layouts "
+                         "(the GEMM alone: operands quantised offline, MN-major ones stored transposed)"),
+    "k_grouped": dict(kind="kgrouped", G=8, shapes=[(4096, 7168), (7168, 2048)], with_c=False,
+                      desc="K-grouped TN FP8 GEMM (MoE weight gradient), G=8 groups of U{2048..6144} tokens "
+                           "padded to 128, (M,N) in {(4096,7168),(7168,2048)}, fp32 D; step = per-channel casts "
+                           "of both token-major operands + the GEMM"),
 }
 METRIC = "FP8 block-scaled GEMM TFLOPS on 1×B200; % of FP8 peak / HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -193,22 +205,42 @@ class ClockSampler:
 
 def make_problems(wl):
     """Host-side problems of a workload (bf16 bit patterns from the seeded generator)."""
+    import numpy as np
+
     from moe_grouped_gemm_sm_b200 import synth
     probs = []
-    for i, (N, K) in enumerate(wl["shapes"]):
+    items = [(i, N, K, lay) for i, (N, K) in enumerate(wl["shapes"]) for lay in wl.get("layouts", ("nt",))]
+    for i, N, K, lay in items:
         kind = wl["kind"]
-        p = dict(kind=kind, N=N, K=K, with_c=wl["with_c"], salt=100 + i)
-        if kind == "dense":
+        p = dict(kind=kind, N=N, K=K, with_c=wl["with_c"], salt=100 + i, ue8m0=wl.get("ue8m0", False))
+        if kind == "layout":
+            x, w, c = synth.dense_inputs(wl["M"], N, K, wl["with_c"], salt=100 + i)
+            p.update(rows=wl["M"], G=1, x=x, w=w, c=c, valid_rows=wl["M"], lay=lay)
+        elif kind == "kgrouped":
+            # (N, K) of the entry are the gradient's (M, N); the K dimension is the tokens
+            M_, N_ = N, K
+            m, _ = synth.contiguous_layout(wl["G"], salt=100 + i)
+            ks = [int((v + 127) // 128 * 128) for v in m]
+            T = sum(ks)
+            dy = synth.normal_bf16(synth.seed_for(synth.BASE_SEED, synth.STREAM_A, 100 + i), (T, M_))
+            xx = synth.normal_bf16(synth.seed_for(synth.BASE_SEED, synth.STREAM_B, 100 + i), (T, N_))
+            p.update(N=N_, K=T, rows=M_, G=wl["G"], x=dy, w=xx, c=None, ks=ks, valid_rows=M_)
+        elif kind == "dense":
             x, w, c = synth.dense_inputs(wl["M"], N, K, wl["with_c"], salt=100 + i)
             p.update(rows=wl["M"], G=1, x=x, w=w, c=c, valid_rows=wl["M"])
         elif kind == "contiguous":
+            # the routed tokens arrive in a seeded shuffled order; the step's cast writes each
+            # one to its row of the expert-grouped layout (dst), as the MoE dispatch does
             m, layout, x, w = synth.contiguous_inputs(wl["G"], N, K, salt=100 + i)
-            p.update(rows=layout.shape[0], G=wl["G"], x=x, w=w, c=None, layout=layout, valid_rows=int(m.sum()))
+            rows = np.nonzero(layout >= 0)[0].astype(np.int32)
+            dst = rows[np.random.default_rng(100 + i).permutation(rows.size)]
+            p.update(rows=layout.shape[0], G=wl["G"], x=np.ascontiguousarray(x[dst]), w=w, c=None, layout=layout,
+                     valid_rows=int(m.sum()), dst=dst)
         else:
             mm, x, w = synth.masked_inputs(wl["G"], wl["M_max"], N, K, salt=100 + i)
             p.update(rows=wl["M_max"], G=wl["G"], x=x, w=w, c=None, masked_m=mm, valid_rows=int(mm.sum()),
                      expected_m=wl["expected_m"])
-        p["flops"] = 2.0 * p["valid_rows"] * N * K
+        p["flops"] = 2.0 * p["valid_rows"] * p["N"] * p["K"]
         p["bytes"] = algorithmic_bytes(p)
         probs.append(p)
     return probs
@@ -219,8 +251,12 @@ def algorithmic_bytes(p):
     weights, fp32 scales, the D rows it must write (and C), the grouped layout or masked_m."""
     N, K, G = p["N"], p["K"], p["G"]
     kb, nb = K // 128, (N + 127) // 128
+    if p["kind"] == "kgrouped":                       # A [T,M], B [T,N], per-channel scales, fp32 D
+        M, T = p["rows"], K
+        pad4 = lambda v: (v + 3) // 4 * 4
+        return T * M + T * N + 4 * (T // 128) * (pad4(M) + pad4(N)) + 4 * G * M * N
     w = G * N * K + 4 * G * nb * kb
-    if p["kind"] == "dense":
+    if p["kind"] in ("dense", "layout"):
         M = p["rows"]
         return M * K + 4 * M * kb + w + 2 * M * N * (2 if p["with_c"] else 1)
     if p["kind"] == "contiguous":
@@ -244,7 +280,14 @@ def fp8_tensor_peak(peaks, clocks):
 
 
 def cast_bytes(p):
-    """Per-token cast of all activation rows: 2 B read and 1 B written per element, plus scales."""
+    """Per-token cast of all activation rows: 2 B read and 1 B written per element, plus scales
+    (K-grouped: the per-channel casts of both token-major operands; the layout workload: none)."""
+    if p["kind"] == "layout":
+        return 0
+    if p["kind"] == "kgrouped":
+        return 3 * p["K"] * (p["rows"] + p["N"]) + 4 * (p["K"] // 128) * (p["rows"] + p["N"])
+    if p["kind"] == "contiguous":                    # the routed tokens only
+        return 3 * p["valid_rows"] * p["K"] + 4 * p["valid_rows"] * (p["K"] // 128)
     rows = p["rows"] * (p["G"] if p["kind"] == "masked" else 1)
     return 3 * rows * p["K"] + 4 * rows * (p["K"] // 128)
 
@@ -264,7 +307,20 @@ SUB_WORKLOADS = [
     ("decode128_warm", "decode128", "warm"),
     ("contiguous", "contiguous", None),
     ("masked", "masked", None),
+    ("prefill_ue8m0", "prefill_ue8m0", None),
+    ("layouts", "layouts", None),
+    ("k_grouped", "k_grouped", None),
 ]
+
+
+def _json_default(o):
+    """numpy scalars and arrays in the result line become plain numbers and lists."""
+    import numpy as np
+    if isinstance(o, np.ndarray):
+        return o.tolist()
+    if isinstance(o, np.generic):
+        return o.item()
+    raise TypeError(f"not serialisable: {type(o).__name__}")
 
 
 def source_digest():
@@ -320,13 +376,38 @@ class CudaArm:
         probs = make_problems(wl)
         wc_ms = []
         for p in probs:
-            key = (p["kind"], p["salt"], p["N"], p["K"], p["G"])
+            if p["kind"] == "kgrouped":
+                T, M, N = p["K"], p["rows"], p["N"]
+                pad4 = lambda v: (v + 3) // 4 * 4
+                p["a"], p["bx"] = self.bf16(p["x"]), self.bf16(p["w"])
+                p["aq"] = torch.empty((T, M), dtype=torch.uint8, device=dev)
+                p["bq"] = torch.empty((T, N), dtype=torch.uint8, device=dev)
+                p["sfa"] = torch.zeros((T // 128, pad4(M)), dtype=torch.float32, device=dev)
+                p["sfb"] = torch.zeros((T // 128, pad4(N)), dtype=torch.float32, device=dev)
+                p["d"] = torch.zeros((p["G"], M, N), dtype=torch.float32, device=dev)
+                p["ks_dev"] = torch.tensor(p["ks"], dtype=torch.int32, device=dev)
+                p["ks_c"] = (ctypes.c_int * len(p["ks"]))(*p["ks"])
+                p["launches"] = 3
+                continue
+            key = (p["kind"], p["salt"], p["N"], p["K"], p["G"], p["ue8m0"])
             if key not in self.weights:
                 w_dev = self.bf16(p["w"])
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                ops.cast_per_block(w_dev)                             # warm the weight cast once
+                if p["ue8m0"]:
+                    nb_, kq_ = (p["N"] + 127) // 128, (p["K"] // 128 + 3) // 4
+                    b = torch.empty((p["N"], p["K"]), dtype=torch.uint8, device=dev)
+                    sfb = torch.empty((nb_, kq_), dtype=torch.int32, device=dev)
+
+                    def wcast():
+                        self._lib.dg_cast_fp8_per_block_ue8m0(w_dev, b, sfb, 1, p["N"], p["K"], self.stream)
+                else:
+                    def wcast():
+                        return ops.cast_per_block(w_dev)
+                wcast()                                               # warm the weight cast once
                 e0.record(self.stream)
-                b, sfb = ops.cast_per_block(w_dev)
+                out = wcast()
+                if not p["ue8m0"]:
+                    b, sfb = out
                 e1.record(self.stream)
                 torch.cuda.synchronize(dev)
                 nb, kb = (p["N"] + 127) // 128, p["K"] // 128
@@ -339,20 +420,51 @@ class CudaArm:
             batch = p["G"] if p["kind"] == "masked" else 1
             p["batch"] = batch
             p["aq"] = torch.empty(p["a"].shape, dtype=torch.uint8, device=dev)
-            p["sfa"] = torch.empty((batch, p["K"] // 128, (p["rows"] + 3) // 4 * 4), dtype=torch.float32, device=dev)
+            if p["ue8m0"]:
+                p["sfa"] = torch.zeros(((p["K"] // 128 + 3) // 4, (p["rows"] + 3) // 4 * 4), dtype=torch.int32,
+                                       device=dev)
+            else:
+                p["sfa"] = torch.empty((batch, p["K"] // 128, (p["rows"] + 3) // 4 * 4), dtype=torch.float32,
+                                       device=dev)
             dshape = (p["G"], p["rows"], p["N"]) if p["kind"] == "masked" else (p["rows"], p["N"])
             p["d"] = torch.zeros(dshape, dtype=torch.bfloat16, device=dev)
             if p["kind"] == "contiguous":
                 p["gl"] = torch.from_numpy(p["layout"]).to(dev)
+                p["dst_dev"] = torch.from_numpy(p["dst"]).to(dev)
+                p["aq"] = torch.zeros((p["rows"], p["K"]), dtype=torch.uint8, device=dev)
+                p["sfa"] = torch.zeros((1, p["K"] // 128, (p["rows"] + 3) // 4 * 4), dtype=torch.float32, device=dev)
             if p["kind"] == "masked":
                 p["mm"] = torch.from_numpy(p["masked_m"]).to(dev)
+            p["launches"] = 2
+            if p["kind"] == "layout":
+                # operands quantised once (untimed), stored in the layout's order
+                self.launch_cast(dict(p, kind="dense"), self.stream.cuda_stream)
+                if p["lay"][0] == "t":
+                    p["aq"] = p["aq"].t().contiguous()
+                if p["lay"][1] == "n":
+                    p["b"] = p["b"].t().contiguous()
+                p["launches"] = 1
         torch.cuda.synchronize(dev)
         return probs, wc_ms
 
     # ---- launches through the C ABI (the same calls a user makes) ----
     def launch_cast(self, p, sptr):
-        rc = self.L.dg_cast_fp8_per_token(p["a"].data_ptr(), p["aq"].data_ptr(), p["sfa"].data_ptr(), p["batch"],
-                                          p["rows"], p["K"], sptr)
+        if p["kind"] == "layout":                           # operands were quantised offline
+            return
+        if p["kind"] == "kgrouped":
+            for x, q, sf, C in ((p["a"], p["aq"], p["sfa"], p["rows"]), (p["bx"], p["bq"], p["sfb"], p["N"])):
+                rc = self.L.dg_cast_fp8_per_channel(x.data_ptr(), q.data_ptr(), sf.data_ptr(), p["K"], C, sptr)
+                if rc:
+                    raise self._lib.DgError("dg_cast_fp8_per_channel", rc)
+            return
+        if p["kind"] == "contiguous":                       # the MoE dispatch: cast into the grouped layout
+            rc = self.L.dg_cast_fp8_per_token_scatter(p["a"].data_ptr(), p["dst_dev"].data_ptr(), p["aq"].data_ptr(),
+                                                      p["sfa"].data_ptr(), p["valid_rows"], p["rows"], p["K"], sptr)
+            if rc:
+                raise self._lib.DgError("dg_cast_fp8_per_token_scatter", rc)
+            return
+        f = self.L.dg_cast_fp8_per_token_ue8m0 if p.get("ue8m0") else self.L.dg_cast_fp8_per_token
+        rc = f(p["a"].data_ptr(), p["aq"].data_ptr(), p["sfa"].data_ptr(), p["batch"], p["rows"], p["K"], sptr)
         if rc:
             raise self._lib.DgError("dg_cast_fp8_per_token", rc)
 
@@ -362,8 +474,17 @@ class CudaArm:
         def ptr(t):
             return t.data_ptr() if t is not None else None
         if p["kind"] == "dense":
-            rc = L.dg_fp8_gemm_nt(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]), ptr(p["cd"]), ptr(p["d"]),
-                                  p["rows"], p["N"], p["K"], sptr)
+            f = L.dg_fp8_gemm_nt_ue8m0 if p.get("ue8m0") else L.dg_fp8_gemm_nt
+            rc = f(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]), ptr(p["cd"]), ptr(p["d"]), p["rows"], p["N"],
+                   p["K"], sptr)
+        elif p["kind"] == "layout":
+            f = getattr(L, "dg_fp8_gemm_" + p["lay"])
+            rc = f(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]), ptr(p["cd"]), ptr(p["d"]), p["rows"],
+                   p["N"], p["K"], sptr)
+        elif p["kind"] == "kgrouped":
+            rc = L.dg_k_grouped_fp8_gemm_tn_contiguous(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["bq"]), ptr(p["sfb"]), None,
+                                                       ptr(p["d"]), ctypes.cast(p["ks_c"], ctypes.c_void_p),
+                                                       ptr(p["ks_dev"]), p["G"], p["rows"], p["N"], sptr)
         elif p["kind"] == "contiguous":
             rc = L.dg_m_grouped_fp8_gemm_nt_contiguous(ptr(p["aq"]), ptr(p["sfa"]), ptr(p["b"]), ptr(p["sfb"]),
                                                        ptr(p["cd"]), ptr(p["d"]), ptr(p["gl"]), p["rows"], p["N"],
@@ -454,7 +575,7 @@ class CudaArm:
         del g_step, g_ev
         return dict(local_ms=local_ms, cast_ms=[statistics.fmean(v) for v in cast_t],
                     gemm_ms=[statistics.fmean(v) for v in gemm_t], clocks=clk.summary(), l2=l2,
-                    launches_per_step=2 * len(probs) + (1 if flush is not None else 0))
+                    launches_per_step=sum(p["launches"] for p in probs) + (1 if flush is not None else 0))
 
 
 L2_TEXT = {"flush": "256 MB L2-flushing write at the start of every step (cold weights)",
@@ -479,7 +600,7 @@ def roofline_of(probs, t, workload):
         t_tc = p["flops"] / (fp8_peak * 1e12)
         t_hbm = p["bytes"] / (hbm * 1e9)
         t_roof_total += max(t_tc, t_hbm)
-        per_problem.append({"N": p["N"], "K": p["K"], "rows": p["rows"], "G": p["G"],
+        per_problem.append({"N": p["N"], "K": p["K"], "rows": p["rows"], "G": p["G"], "layout": p.get("lay", "nt"),
                             "kernel": p.get("kernel", ""), "flops": p["flops"], "bytes": p["bytes"],
                             "gemm_us": round(gm * 1e3, 2),
                             "tflops": round(p["flops"] / (gm * 1e-3) / 1e12, 1),
@@ -624,7 +745,7 @@ def run_cuda(args):
         result["workloads"] = subs
 
     if rank == 0:
-        print(json.dumps(result), flush=True)
+        print(json.dumps(result, default=_json_default), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
