@@ -43,8 +43,9 @@
  *    the stated bound): DG_FORCE_PAIR=0|1 (CTA pairs for the tile GEMM), DG_FORCE_BN=128|256,
  *    DG_FORCE_SWAP=0|1 (few-row kernels off for M <= 128, or on for the masked layout),
  *    DG_FEW_ROW=streamk|cluster, DG_SPLITK_S=1|2|3|4|6|8|16 (cluster size), DG_ONE_ISSUER=1
- *    (one MMA-issuing thread per CTA instead of two). Debug only:
- *    DG_TEST_SKIP_RELEASE=1|2|3 makes one kernel withhold barrier arrives or partial flags,
+ *    (one MMA-issuing thread per CTA instead of two), DG_TAIL_SPLIT=0|2..64 (the dense tile
+ *    GEMM's last-wave split off, or S pieces per last-wave tile). Debug only:
+ *    DG_TEST_SKIP_RELEASE=1|2|3|4 makes one kernel withhold barrier arrives or partial flags,
  *    so that a wait runs out of time (failure tests).
  */
 #ifndef DG_H
@@ -81,9 +82,14 @@ typedef enum dg_status {
  *   - with few 128-column tiles (at most 64) and K <= 8192, over a thread-block cluster per
  *     tile, whose partial sums meet in distributed shared memory (no scratch at all);
  *   - otherwise over every SM (stream-K), whose partial sums meet in a library-owned
- *     workspace of the (device, stream) pair, allocated (cudaMalloc, sm_count x 64 KB) by
- *     the pair's first such call and kept until the process ends; a first call made under
- *     CUDA-graph capture cannot allocate and computes with the tile kernel instead.
+ *     workspace of the (device, stream) pair, allocated (cudaMalloc, sm_count x 128 KB plus
+ *     the flags) by the pair's first call that wants it and kept until the process ends; a
+ *     first call made under CUDA-graph capture cannot allocate and computes with the tile
+ *     kernel instead.
+ * For M > 128 (the persistent tile kernel), when the tiles do not fill a whole number of
+ * waves of resident CTAs, the last wave's tiles are cut along K into pieces run at once on
+ * otherwise idle SMs, whose partial sums meet in the same workspace (in a fixed order); without
+ * a workspace (a first call under graph capture) the last wave runs whole.
  * Every choice gives the same result within the stated bound, and each is deterministic. */
 DG_API dg_status dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const float *sfb,
                          const void *c, void *d, int M, int N, int K, void *stream);
@@ -184,7 +190,8 @@ DG_API dg_status dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float 
  *   b   e4m3 [G,N,K];                  sfb fp32 [G][Nb][Kb]
  *   masked_m  int32 [G] on the device, read by the kernel (values > M_max are clamped to
  *       M_max and set the device error word; negative values count as 0).
- *   expected_m  host-side hint of the typical masked_m, used only to choose tile shapes.
+ *   expected_m  host-side hint of the typical masked_m, used only to choose tile shapes:
+ *       128-row tiles when expected_m <= 128, 256-row CTA-pair tiles above (0 = use M_max).
  *   c   bf16 [G,M_max,N] or NULL;      d bf16 [G,M_max,N].
  * Rows r >= masked_m[g] of D are never written and their A rows never reach D. */
 DG_API dg_status dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void *b,
@@ -265,8 +272,11 @@ DG_API dg_status dg_get_device_error(void *stream);
 DG_API const char *dg_status_string(dg_status status);
 
 /* Name of the GEMM kernel that the calling thread's last GEMM call launched ("" before the
- * first): "gemm_kernel", "gemm_kernel (CTA pairs)", "gemm_swap_kernel (stream-K)" or
- * "gemm_splitk_kernel (cluster split-K)". For benchmarks and profiles; static storage. */
+ * first): "gemm_kernel", "gemm_kernel (CTA pairs)", "gemm_kernel (last-wave split S)" or
+ * "gemm_kernel (CTA pairs, last-wave split S)" when the last wave's tiles were cut into S K
+ * pieces, "gemm_swap_kernel (stream-K)",
+ * "gemm_splitk_kernel (cluster split-K)" or "gemm_bs_kernel (UE8M0 block-scaled MMA)". For
+ * benchmarks and profiles; valid until the thread's next GEMM call. */
 DG_API const char *dg_last_kernel(void);
 
 /* Bytes of device memory the library has allocated with cudaMalloc so far, over all devices

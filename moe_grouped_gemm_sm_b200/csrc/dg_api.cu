@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -37,6 +38,7 @@ std::atomic<long long> g_allocated{0};
 
 // Name of the GEMM kernel the calling thread's last GEMM call launched; dg_last_kernel().
 thread_local const char *t_last_kernel = "";
+thread_local char t_kernel_name[96];   // names with a number in them (the last-wave split)
 
 struct DeviceInfo {
     std::atomic<bool> ready{false};
@@ -209,17 +211,35 @@ bool use_streamk(int groups, int m_tiles, int N, int K) {
     return tiles > 64 || K / 128 > 64;
 }
 
+// Last-wave split of the dense tile GEMM for tests and experiments (DG_TAIL_SPLIT=0: off,
+// 2..64: pieces per last-wave tile, capped by the grid and by K); -1 = cost model.
+int forced_tail_split() {
+    static std::atomic<int> cached{-2};
+    int v = cached.load();
+    if (v == -2) {
+        v = -1;
+        if (const char *s = std::getenv("DG_TAIL_SPLIT")) {
+            v = std::atoi(s);
+            if (v != 0 && (v < 2 || v > 64)) v = -1;
+        }
+        cached.store(v);
+    }
+    return v;
+}
+
 // Failure tests only (DG_TEST_SKIP_RELEASE): 1 = the tile GEMM withholds one TMEM-buffer
 // release, 2 = the cluster split-K GEMM withholds one partial-push arrive, 3 = the process's
-// first two stream-K launches have their odd-numbered CTAs withhold their partial flags. A bounded wait
-// then runs out of time and reports DG_ERR_TIMEOUT without faulting. 0 = off.
+// first two stream-K launches have their odd-numbered CTAs withhold their partial flags, 4 = the
+// process's first tile-GEMM launch with a last-wave split has its piece CTAs withhold their
+// partial flags. A bounded wait then runs out of time and reports DG_ERR_TIMEOUT without
+// faulting. 0 = off.
 int test_skip_release() {
     static std::atomic<int> cached{-1};
     int v = cached.load();
     if (v < 0) {
         const char *s = std::getenv("DG_TEST_SKIP_RELEASE");
         v = s ? std::atoi(s) : 0;
-        if (v != 1 && v != 2 && v != 3) v = 0;
+        if (v < 1 || v > 4) v = 0;
         cached.store(v);
     }
     return v;
@@ -228,6 +248,11 @@ int test_skip_release() {
 bool test_skip_streamk_flags() {
     static std::atomic<int> launches{0};
     return test_skip_release() == 3 && launches.fetch_add(1) < 2;
+}
+
+bool test_skip_tail_flags() {
+    static std::atomic<int> launches{0};
+    return test_skip_release() == 4 && launches.fetch_add(1) < 1;
 }
 
 // Encodes a tiled tensor map. dims/box are innermost first; strides (bytes) for dims 1..rank-1.
@@ -340,11 +365,101 @@ struct KernelInfo {
     int max_clusters = 0;
 };
 
-template <int BN, int STAGES, int KIND, bool PAIR, bool A_MN = false, bool B_MN = false>
-dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p, int tiles, const DeviceInfo *di, cudaStream_t st) {
+// Flag workspace of a (device, stream): fp32 partials, one flag per slot and the two words of
+// the launch epoch (all zero when allocated). Shared by the stream-K few-row kernel (partials
+// [CTA][128][128], flags [CTA]) and the tile GEMM's last-wave split (partials [slot][128][256],
+// flags [slot][8 math warps]); both follow the same ticket protocol, so their flags never
+// need clearing. One per (device, stream), so that launches on different streams never share
+// flags; allocated on a stream's first call that wants it, which must not be under graph capture
+// (the call then goes without: the tile kernel without the split, the few-row GEMM through the
+// tile kernel).
+struct StreamWorkspace {
+    int dev = -1;
+    cudaStream_t stream = nullptr;
+    float *ws = nullptr;    // sm_count x 128 KB
+    int *flags = nullptr;   // [slots] flags, then the epoch words
+    int slots = 0;          // 8 x sm_count
+};
+std::vector<StreamWorkspace> g_stream_ws;
+
+bool stream_workspace(int dev, int sm_count, cudaStream_t st, StreamWorkspace *out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (const StreamWorkspace &w : g_stream_ws)
+        if (w.dev == dev && w.stream == st) {
+            *out = w;
+            return true;
+        }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return false;
+    StreamWorkspace w;
+    w.dev = dev;
+    w.stream = st;
+    w.slots = 8 * sm_count;
+    const size_t ws_bytes = static_cast<size_t>(sm_count) * 128 * 256 * sizeof(float);
+    const size_t flag_bytes = static_cast<size_t>(w.slots + 2) * sizeof(int);
+    if (cudaMalloc(&w.ws, ws_bytes) != cudaSuccess) return false;
+    if (cudaMalloc(&w.flags, flag_bytes) != cudaSuccess) {
+        cudaFree(w.ws);
+        return false;
+    }
+    if (cudaMemset(w.flags, 0, flag_bytes) != cudaSuccess) {
+        cudaFree(w.ws);
+        cudaFree(w.flags);
+        return false;
+    }
+    g_allocated += static_cast<long long>(ws_bytes + flag_bytes);
+    g_stream_ws.push_back(w);
+    *out = w;
+    return true;
+}
+
+// Last-wave split plan of a dense NT launch of `tiles` tiles over `units` persistent CTAs
+// (pairs): the R = tiles mod units tiles of the last wave are cut along K into S pieces, run
+// by a second launch, when that shortens the last wave. Cost model in K-block times (measured
+// on B200, 256 x 256 pair tiles): the split saves Kb·(1 - 1/S), costs ~2.7 per extra piece
+// (a partial written and read through L2) and a fixed ~20 (the second launch's pipeline fill,
+// the exchange, the epilogue; ~26 when whole waves run before it). The best S of at most
+// units / R pieces, at least 2 K blocks each, if it saves more than 5. No workspace (a first
+// call under graph capture): no split.
+void plan_tail(dg::GemmParams &q, int tiles, int units, float *ws, int *flags, unsigned *epoch) {
+    q.tail_first = tiles;
+    q.tail_s = 1;
+    q.tail_units = 0;
+    const int forced = forced_tail_split();
+    if (!ws || forced == 0 || units <= 0) return;
+    const int F = tiles / units, R = tiles - F * units;
+    if (R == 0) return;
+    const int s_max = std::min(units / R, q.Kb / 2);
+    int S = 1;
+    if (forced > 0) {
+        S = std::min(forced, s_max);
+    } else {
+        const double fixed = F > 0 ? 26.0 : 20.0;
+        double best = 5.0;
+        for (int s = 2; s <= s_max; ++s) {
+            const double gain = q.Kb * (1.0 - 1.0 / s) - 2.7 * (s - 1) - fixed;
+            if (gain > best) {
+                best = gain;
+                S = s;
+            }
+        }
+    }
+    if (S < 2) return;
+    q.tail_first = F * units;
+    q.tail_s = S;
+    q.tail_units = R * S;
+    q.ws = ws;
+    q.flags = flags;
+    q.epoch = epoch;
+    q.test_skip_tail = test_skip_tail_flags();
+}
+
+template <int BN, int STAGES, int KIND, bool PAIR, bool A_MN = false, bool B_MN = false, bool TAIL = false>
+dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p_in, int tiles, const DeviceInfo *di,
+                      cudaStream_t st, float *ws = nullptr, int *flags = nullptr, unsigned *epoch = nullptr) {
     constexpr bool PAIR_LIST = PAIR && KIND == dg::KIND_CONTIGUOUS;
     using L = dg::GemmLayout<BN, STAGES, PAIR, PAIR_LIST, KIND == dg::KIND_KGROUPED>;
-    auto kern = dg::gemm_kernel<BN, STAGES, KIND, PAIR, A_MN, B_MN>;
+    auto kern = dg::gemm_kernel<BN, STAGES, KIND, PAIR, A_MN, B_MN, TAIL>;
     static KernelInfo info[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
@@ -366,6 +481,27 @@ dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p, int tiles, co
         }
     }
     const int units = PAIR ? ki.max_clusters : di->sm_count;
+    dg::GemmParams p = p_in;
+    if constexpr (!TAIL && KIND == dg::KIND_DENSE && !A_MN && !B_MN) {
+        plan_tail(p, tiles, units, ws, flags, epoch);
+        if (p.tail_s > 1) {
+            // the whole waves (if any) in this kernel, then the last wave's pieces in the TAIL
+            // instantiation, launched behind it on the stream
+            if (p.tail_first > 0) {
+                p.tail_early = 1;
+                p.num_tiles = p.tail_first;
+                cfg.gridDim = dim3(PAIR ? 2 * units : units, 1, 1);
+                const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mp.a, mp.b, mp.sfa, mp.c, mp.d, mp.sfb, p);
+                if (e != cudaSuccess) return from_cuda(e);
+            }
+            const dg_status r = launch_gemm<BN, STAGES, KIND, PAIR, A_MN, B_MN, true>(mp, p, p.tail_units, di, st);
+            std::snprintf(t_kernel_name, sizeof(t_kernel_name),
+                          PAIR ? "gemm_kernel (CTA pairs, last-wave split %d)" : "gemm_kernel (last-wave split %d)",
+                          p.tail_s);
+            t_last_kernel = t_kernel_name;
+            return r;
+        }
+    }
     const int n_units = tiles < units ? tiles : units;
     if (n_units <= 0) return DG_OK;
     cfg.gridDim = dim3(PAIR ? 2 * n_units : n_units, 1, 1);
@@ -379,7 +515,8 @@ dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p, int tiles, co
 // N <= 128. Stages fill the shared-memory budget.
 template <int KIND, bool A_MN = false, bool B_MN = false>
 dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *sfb, const void *c, void *d,
-                   const int32_t *layout, const int32_t *masked_m, int rows, int N, int K, int G, cudaStream_t st) {
+                   const int32_t *layout, const int32_t *masked_m, int rows, int N, int K, int G, cudaStream_t st,
+                   int expected_m = 0) {
     const DeviceInfo *di = nullptr;
     dg_status s = device_info(&di);
     if (s != DG_OK) return s;
@@ -405,7 +542,12 @@ dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *
     const int fbn = forced_bn();
     const int bn = fbn ? fbn : (N > 128 ? 256 : 128);
     const int fpair = forced_pair();
-    bool pair = fpair >= 0 ? fpair == 1 : rows > 128;
+    // masked: the expected rows per expert choose the tile height (CTA pairs of 256 rows only
+    // when a typical expert fills more than one 128-row tile; measured on G = 16 experts of
+    // N x K = 4096 x 7168 and 7168 x 2048: expected_m 32 and 96 run 23 % faster on 128-row
+    // tiles, expected_m 192 within 3 % either way)
+    const int hint_rows = KIND == dg::KIND_MASKED && expected_m > 0 ? expected_m : rows;
+    bool pair = fpair >= 0 ? fpair == 1 : hint_rows > 128;
     if (KIND == dg::KIND_CONTIGUOUS && rows / 128 > dg::MAX_PAIR_BLOCKS) pair = false;
     if (bn != 256) pair = false;                       // pairs are built for 256-column tiles
     GemmMaps mp;
@@ -428,11 +570,23 @@ dg_status run_gemm(const void *a, const float *sfa, const void *b, const float *
     om.b_mn = B_MN;
     if (!build_maps(mp, a, sfa, b, c, d, rows, N, K, G, b_rows, batched, p.cd_blocks ? bn / 128 : 0, om))
         return DG_ERR_INVALID_ARG;
-    if (pair) {
-        return launch_gemm<256, 4, KIND, true, A_MN, B_MN>(mp, p, tiles, di, st);
+    // dense: the stream's flag workspace for a last-wave split (none: no split)
+    float *ws = nullptr;
+    int *flags = nullptr;
+    unsigned *epoch = nullptr;
+    StreamWorkspace w;
+    int dev = 0;
+    if (KIND == dg::KIND_DENSE && forced_tail_split() != 0 && cudaGetDevice(&dev) == cudaSuccess &&
+        stream_workspace(dev, di->sm_count, st, &w)) {
+        ws = w.ws;
+        flags = w.flags;
+        epoch = reinterpret_cast<unsigned *>(w.flags + w.slots);
     }
-    if (bn == 256) return launch_gemm<256, 3, KIND, false, A_MN, B_MN>(mp, p, tiles, di, st);
-    return launch_gemm<128, 5, KIND, false, A_MN, B_MN>(mp, p, tiles, di, st);
+    if (pair) {
+        return launch_gemm<256, 4, KIND, true, A_MN, B_MN>(mp, p, tiles, di, st, ws, flags, epoch);
+    }
+    if (bn == 256) return launch_gemm<256, 3, KIND, false, A_MN, B_MN>(mp, p, tiles, di, st, ws, flags, epoch);
+    return launch_gemm<128, 5, KIND, false, A_MN, B_MN>(mp, p, tiles, di, st, ws, flags, epoch);
 }
 
 // K-grouped TN GEMM (the MoE weight gradient): A [sum_K][M] and B [sum_K][N], both MN-major,
@@ -536,51 +690,6 @@ bool build_swap_maps(SwapMaps &mp, const void *a, const float *sfa, const void *
     return true;
 }
 
-// Stream-K workspace of the few-row kernel: fp32 partials [slots][128][128], one flag per
-// slot and the two words of the launch epoch (all zero when allocated). One per (device,
-// stream), so that launches on different streams never share flags; allocated on a stream's
-// first few-row call, which must not be under graph capture (the call then takes the tile
-// kernel, which needs no workspace).
-struct SwapWorkspace {
-    int dev = -1;
-    cudaStream_t stream = nullptr;
-    float *ws = nullptr;
-    int *flags = nullptr;   // [slots] flags, then the epoch words
-    int slots = 0;
-};
-std::vector<SwapWorkspace> g_swap_ws;
-
-bool swap_workspace(int dev, int sm_count, cudaStream_t st, SwapWorkspace *out) {
-    std::lock_guard<std::mutex> lk(g_mu);
-    for (const SwapWorkspace &w : g_swap_ws)
-        if (w.dev == dev && w.stream == st) {
-            *out = w;
-            return true;
-        }
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return false;
-    SwapWorkspace w;
-    w.dev = dev;
-    w.stream = st;
-    w.slots = sm_count;
-    const size_t ws_bytes = static_cast<size_t>(sm_count) * 128 * 128 * sizeof(float);
-    const size_t flag_bytes = static_cast<size_t>(sm_count + 2) * sizeof(int);
-    if (cudaMalloc(&w.ws, ws_bytes) != cudaSuccess) return false;
-    if (cudaMalloc(&w.flags, flag_bytes) != cudaSuccess) {
-        cudaFree(w.ws);
-        return false;
-    }
-    if (cudaMemset(w.flags, 0, flag_bytes) != cudaSuccess) {
-        cudaFree(w.ws);
-        cudaFree(w.flags);
-        return false;
-    }
-    g_allocated += static_cast<long long>(ws_bytes + flag_bytes);
-    g_swap_ws.push_back(w);
-    *out = w;
-    return true;
-}
-
 template <int TN, int STAGES, int KIND>
 dg_status launch_swap(const SwapMaps &mp, const dg::SwapParams &p, long long tiles, const DeviceInfo *di,
                       cudaStream_t st) {
@@ -656,8 +765,8 @@ dg_status run_swap(const void *a, const float *sfa, const void *b, const float *
     if (s != DG_OK) return s;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_CUDA;
-    SwapWorkspace w;
-    if (!swap_workspace(dev, di->sm_count, st, &w)) return DG_ERR_UNSUPPORTED;
+    StreamWorkspace w;
+    if (!stream_workspace(dev, di->sm_count, st, &w)) return DG_ERR_UNSUPPORTED;
     return run_swap_with<KIND>(a, sfa, b, sfb, c, d, masked_m, expected_m, rows, N, K, G, st, di, w.ws, w.flags,
                                w.slots);
 }
@@ -951,7 +1060,7 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const
     dg_status s = check_gemm_common(a, sfa, b, sfb, c, d, N, K);
     if (s != DG_OK) return s;
     if (M_max == 0) return DG_OK;
-    if (forced_swap() == 1) {   // the pair kernel streams the masked page shapes faster
+    if (forced_swap() == 1) {   // the tile kernels stream the masked page shapes faster
         const dg_status r = use_streamk(G, 1, N, K)
                                 ? run_swap<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, masked_m, expected_m, M_max, N, K,
                                                             G, static_cast<cudaStream_t>(stream))
@@ -960,7 +1069,7 @@ dg_status dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const
         if (r != DG_ERR_UNSUPPORTED) return r;
     }
     return run_gemm<dg::KIND_MASKED>(a, sfa, b, sfb, c, d, nullptr, masked_m, M_max, N, K, G,
-                                     static_cast<cudaStream_t>(stream));
+                                     static_cast<cudaStream_t>(stream), expected_m);
 }
 
 dg_status dg_transform_sf(const float *sf_kmajor, float *sf_mnmajor, int batch, int MN, int Kb, void *stream) {

@@ -22,11 +22,12 @@
 //               ring's barriers.)
 //   warps 1, 3  (leader only) the MMA issuers, one thread each: warp 1 issues the even K
 //               blocks, warp 3 the odd ones, each tcgen05.mma kind::f8f6f4, four K=32 steps per
-//               K block, into its own TMEM buffer, and commits the stage (empty) and the buffer
-//               (tfull) — to both CTAs of a pair. A commit holds back the MMAs its thread issues
-//               after it until the committed ones are done (~800 cycles per K block with one
-//               issuer, measured); MMAs of the other thread keep the tensor pipe busy meanwhile,
-//               so with two issuers a K block costs its nominal ~540 cycles. Two issuers need an
+//               K block, into its own TMEM buffer, and commits the buffer (tfull) — to both CTAs
+//               of a pair; the math warps hand the operand stage back (empty) once they have
+//               seen that commit, which spares the issuer a second commit per K block. A commit
+//               holds back the MMAs its thread issues after it until the committed ones are done
+//               (~800 cycles per K block with one issuer, measured); MMAs of the other thread
+//               keep the tensor pipe busy meanwhile. Two issuers need an
 //               even number of stages and buffers: then every stage and buffer belongs to one
 //               issuer, which waits on its barriers phase after phase. (With an odd count a
 //               stage alternates between the issuers, and one of them could wait for a phase of
@@ -53,6 +54,16 @@
 // expert computes but does not store. Masked: tiles are enumerated per expert over
 // ceil(masked_m[g]/rows per tile) tiles only (likun.im §二 masked_m), and rows >= masked_m[g]
 // are never stored.
+//
+// Last-wave split (dense NT): when the tiles do not fill a whole number of waves of the
+// persistent grid, the main launch runs the whole waves and a second launch of the TAIL
+// instantiation runs the R tiles of the last wave, each cut along K into S pieces on R·S CTAs
+// (pairs) at once. The CTAs of pieces 1..S-1 write their fp32 partials to a global workspace,
+// one flag per math warp; the CTA of piece 0 waits for those flags (bounded), adds the partials
+// in piece order and writes D. A flag holds the ticket of the launch that wrote it (the epoch
+// protocol of the stream-K kernel), so the flags never need clearing. (The split lives in its
+// own instantiation because its code, present but idle in the main kernel, measurably slowed
+// the main kernel's K loop.)
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -86,6 +97,14 @@ struct GemmParams {
     const int32_t *grouped_layout;
     const int32_t *masked_m;
     const int32_t *ks;       // K-grouped: tokens of each group (device), multiples of 128
+    // last-wave split (the TAIL kernel): its unit u < tail_units = R·S is piece u % tail_s of
+    // tile tail_first + u / tail_s, the tiles before tail_first being the main launch's
+    int tail_first, tail_s, tail_units;
+    float *ws;               // partials [slot][8 math warps][HALF / 4][32 lanes] float4
+    int *flags;              // [slot][8 math warps] tickets
+    unsigned *epoch;         // [2]: the last finished launch's ticket, finished-CTA count
+    int tail_early;          // TAIL kernel right behind its main kernel: starts without waiting
+    int test_skip_tail;      // failure test only: piece CTAs withhold their partial flags
     __nv_bfloat16 *d;
     float *d32;              // K-grouped: fp32 D [G][M][N]
     const float *c32;        // K-grouped: fp32 C [G][M][N] or NULL (may alias d32)
@@ -128,8 +147,9 @@ struct TileInfo {
     int row0;     // first row (in the group's row space) of this CTA's 128-row block
     int n_blk;
     int g;
-    int kb0;      // first K block (K-grouped: the group's offset; else 0)
-    int nkb;      // K blocks of the tile (K-grouped: the group's; else Kb)
+    int kb0;      // first K block (K-grouped: the group's offset; last-wave piece: its start)
+    int nkb;      // K blocks of the tile (K-grouped: the group's; last-wave piece: its share)
+    int piece;    // last-wave split: piece index (0 writes D); -1 for a whole tile
     bool valid;   // the tile exists (all CTAs of the pair agree)
     bool store;   // this CTA's rows belong to the tile's expert
 };
@@ -166,6 +186,7 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams &p, cons
     ti.g = 0;
     ti.kb0 = 0;
     ti.nkb = p.Kb;
+    ti.piece = -1;
     if (KIND == KIND_KGROUPED) {
         // group-major: every group's tiles (all of them, also for an empty group, whose D is C)
         // before the next group's, rasterised within the group; the K-block offsets of the
@@ -224,6 +245,27 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams &p, cons
         ti.valid = (g >= 0 && g < p.G);
     }
     return ti;
+}
+
+// Work unit w of the persistent loop: a whole tile, or (TAIL kernel) a K piece of a tile.
+template <int KIND, bool PAIR, bool TAIL>
+__device__ __forceinline__ TileInfo decode_unit(int w, const GemmParams &p, const uint16_t *pair_first,
+                                                int num_pairs, uint32_t rank) {
+    if (!TAIL) return decode_tile<KIND, PAIR>(w, p, pair_first, num_pairs, rank);
+    const int r = w / p.tail_s;                  // which last-wave tile
+    const int pc = w - r * p.tail_s;             // which piece of it
+    TileInfo ti = decode_tile<KIND, PAIR>(p.tail_first + r, p, pair_first, num_pairs, rank);
+    ti.kb0 = pc * p.Kb / p.tail_s;
+    ti.nkb = (pc + 1) * p.Kb / p.tail_s - ti.kb0;
+    ti.piece = pc;
+    return ti;
+}
+
+// Ticket of a launch that uses the flag workspace: one past the epoch word, never 0 (flags
+// start out zero). The last CTA of the grid to finish stores it back into the epoch word.
+__device__ __forceinline__ int streamk_ticket(const unsigned *epoch) {
+    const unsigned e = *reinterpret_cast<const volatile unsigned *>(epoch);
+    return static_cast<int>(e + 1u == 0u ? 1u : e + 1u);
 }
 
 // Contiguous layout, pair tiles: one warp lists the first 128-row block of every pair. Pairs
@@ -318,7 +360,7 @@ __device__ __forceinline__ void tmem_ld_wait_regs32(uint32_t (&r)[32]) {
 // layout names of the pages) instead of K-contiguous; tm_a / tm_b then map those arrays and
 // the MMA reads them through MN-major descriptors. tm_sfb (K-grouped only) maps the per-column
 // B scales [Kb][pad4(N)].
-template <int BN, int STAGES, int KIND, bool PAIR, bool A_MN = false, bool B_MN = false>
+template <int BN, int STAGES, int KIND, bool PAIR, bool A_MN = false, bool B_MN = false, bool TAIL = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_c,
@@ -328,6 +370,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     constexpr bool PAIR_LIST = PAIR && KIND == KIND_CONTIGUOUS;
     constexpr bool KGRP = KIND == KIND_KGROUPED;
     static_assert(!(A_MN || B_MN) || KIND == KIND_DENSE || KGRP, "MN-major operands: dense and K-grouped only");
+    static_assert(!TAIL || KIND == KIND_DENSE, "last-wave split: dense only");
+    constexpr bool KSUB = KGRP || TAIL;        // units cover a sub-range of the K blocks
     using L = GemmLayout<BN, STAGES, PAIR, PAIR_LIST, KGRP>;
     constexpr int HALF = L::HALF;
     constexpr int NBUF = L::NBUF;
@@ -345,6 +389,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const float *sfa_ring = reinterpret_cast<const float *>(smem + L::OFF_SFA);   // slots of SF_SLOT floats
     WaitCtx *ctx = reinterpret_cast<WaitCtx *>(smem + L::OFF_MISC);
     int *num_pairs_smem = reinterpret_cast<int *>(smem + L::OFF_MISC + sizeof(WaitCtx));
+    int *ticket_smem = num_pairs_smem + 1;     // last-wave split: this launch's flag ticket
     uint16_t *pair_first = reinterpret_cast<uint16_t *>(smem + L::OFF_PAIRS);
     volatile int *abort_flag = &ctx->abort;
 
@@ -354,13 +399,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const bool leader = rank == 0;
     const int cid = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     const int ncid = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
-    pdl_launch_dependents();
 
     // prologue (overlaps the previous kernel's tail): barriers, descriptors, TMEM
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], 1);   // math warp 4 of this CTA, once the K block's MMAs are done
         }
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(&tfull[b], 1);
@@ -393,12 +437,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tmem_relinquish();
         }
     }
-    pdl_wait();   // from here on global memory may be read and written
+    // Programmatic dependent launch. A kernel waits for its predecessor here (from here on
+    // global memory may be read and written) and only then lets its dependent launch. So a
+    // TAIL kernel launched right behind its main kernel (tail_early), whose tiles and workspace
+    // the main kernel never touches, may start at once, on SMs the main kernel has left:
+    // everything before the main kernel is complete by then. It waits for the main kernel only
+    // before it exits, so that it never completes before it (the next kernel's wait covers
+    // both). A TAIL kernel with no main kernel before it waits here like any other.
+    if (!TAIL || !p.tail_early) pdl_wait();
+    pdl_launch_dependents();
     if (PAIR_LIST && warp == 2) {
         const int np = build_pair_list(p, pair_first, lane);
         if (lane == 0) *num_pairs_smem = np;
     }
     if (KGRP && warp == 2 && lane == 0) build_kgroup_offsets(p, reinterpret_cast<int *>(pair_first));
+    if (TAIL && threadIdx.x == 0) *ticket_smem = streamk_ticket(p.epoch);
     tc_fence_before();
     if (PAIR)
         cluster_sync();
@@ -409,7 +462,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int num_pairs = PAIR_LIST ? *num_pairs_smem : 0;
 
     int num_tiles;
-    if (KIND == KIND_MASKED)
+    if (TAIL)
+        num_tiles = p.tail_units;
+    else if (KIND == KIND_MASKED)
         num_tiles = masked_num_tiles<UNIT>(p);
     else if (PAIR_LIST)
         num_tiles = num_pairs * p.n_blocks;
@@ -436,17 +491,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (stream >= 0) {
             uint32_t it = 0;
             for (int t = cid; t < num_tiles && !*abort_flag; t += ncid) {
-                const TileInfo ti = decode_tile<KIND, PAIR>(t, p, pair_first, num_pairs, rank);
+                const TileInfo ti = decode_unit<KIND, PAIR, TAIL>(t, p, pair_first, num_pairs, rank);
                 if (!ti.valid) {
                     if (stream == 0 && parity == 0 && KIND == KIND_CONTIGUOUS && ti.g >= p.G) report_error(p.err, ERR_DATA);
                     continue;
                 }
                 const int brow = ti.n_blk * BN + static_cast<int>(rank) * L::B_ROWS;
                 const int bz = KGRP ? 0 : ti.g;                    // K-grouped B: one [sum_K, N] array
-                const int nkb = KGRP ? ti.nkb : p.Kb;
+                const int nkb = KSUB ? ti.nkb : p.Kb;
                 for (int kbl = 0; kbl < nkb; ++kbl, ++it) {
                     if (it % nlanes != parity) continue;
-                    const int kb = KGRP ? ti.kb0 + kbl : kbl;      // K block in the operands' K space
+                    const int kb = KSUB ? ti.kb0 + kbl : kbl;      // K block in the operands' K space
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (stream == 0) {
@@ -513,9 +568,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             constexpr uint64_t A_STEP = A_MN ? 256 : 2, B_STEP = B_MN ? 256 : 2;
             uint32_t it = 0;
             for (int t = cid; t < num_tiles && !*abort_flag; t += ncid) {
-                const TileInfo ti = decode_tile<KIND, PAIR>(t, p, pair_first, num_pairs, rank);
+                const TileInfo ti = decode_unit<KIND, PAIR, TAIL>(t, p, pair_first, num_pairs, rank);
                 if (!ti.valid) continue;
-                const int nkb = KGRP ? ti.nkb : p.Kb;
+                const int nkb = KSUB ? ti.nkb : p.Kb;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     if (two && (it & 1u) != mine) continue;
                     const int s = it % STAGES;
@@ -537,13 +592,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         else
                             umma_f8(dt, ad + A_STEP * k, bd + B_STEP * k, IDESC, k > 0 ? 1u : 0u);
                     }
-                    if (PAIR) {
-                        umma_commit_pair(&empty[s], 0x3);
+                    // one commit per K block: the math warps hand the operand stage back once they
+                    // have seen the MMAs complete (a commit costs the issuing thread several
+                    // times what an MMA does)
+                    if (PAIR)
                         umma_commit_pair(&tfull[b], 0x3);
-                    } else {
-                        umma_commit(&empty[s]);
+                    else
                         umma_commit(&tfull[b]);
-                    }
                 }
             }
         }
@@ -558,14 +613,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         uint32_t it = 0, ctile = 0;
         bool ok = true;
         for (int t = cid; t < num_tiles && ok; t += ncid) {
-            const TileInfo ti = decode_tile<KIND, PAIR>(t, p, pair_first, num_pairs, rank);
+            const TileInfo ti = decode_unit<KIND, PAIR, TAIL>(t, p, pair_first, num_pairs, rank);
             if (!ti.valid) continue;
             const int col0 = ti.n_blk * BN + wg * HALF;          // first column of this warp
             const int srow0 = ti.row0 + q * 32;                  // first row of this warp's slab
             const int row = srow0 + lane;                        // this thread's row
             const int nblk = min(col0 / 128, p.Nb - 1);
-            const float *sfb_row = p.sfb + (static_cast<size_t>(ti.g) * p.Nb + nblk) * p.Kb;
-            const bool do_c = !KGRP && p.has_c && ti.store;
+            // (a last-wave piece starts at K block kb0: its window is offset by that)
+            const float *sfb_row = p.sfb + (static_cast<size_t>(ti.g) * p.Nb + nblk) * p.Kb + (TAIL ? ti.kb0 : 0);
+            const bool do_c = !KGRP && p.has_c && ti.store && (!TAIL || ti.piece == 0);   // piece 0 writes D
             if (do_c && lane == 0) {
                 bulk_wait_group_read0();                         // the slab's last store has read it
                 fence_proxy_async_smem();
@@ -589,21 +645,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             // shuffle); sfa of this thread's row from the TMA-filled ring. No global load is left
             // in flight across the loop's release-arrives except a window refill every 32 blocks.
             // (K-grouped: one B scale per column, from the same ring slot as sfa)
-            float sb_win = !KGRP && lane < p.Kb ? __ldg(sfb_row + lane) : 0.f;
-            float sb_nxt = !KGRP && 32 + lane < p.Kb ? __ldg(sfb_row + 32 + lane) : 0.f;
-            const int nkb = KGRP ? ti.nkb : p.Kb;
+            const int nkb = KSUB ? ti.nkb : p.Kb;
+            float sb_win = !KGRP && lane < nkb ? __ldg(sfb_row + lane) : 0.f;
+            float sb_nxt = !KGRP && 32 + lane < nkb ? __ldg(sfb_row + 32 + lane) : 0.f;
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int b = it % NBUF;
                 const uint32_t phb = (it / NBUF) & 1;
                 if (!KGRP && (kb & 31) == 0 && kb > 0) {
                     sb_win = sb_nxt;
-                    sb_nxt = kb + 32 + lane < p.Kb ? __ldg(sfb_row + kb + 32 + lane) : 0.f;
+                    sb_nxt = kb + 32 + lane < nkb ? __ldg(sfb_row + kb + 32 + lane) : 0.f;
                 }
                 const float sb = KGRP ? 1.f : __shfl_sync(0xFFFFFFFFu, sb_win, kb & 31);
                 const int j = it % L::SFS;
                 // every lane waits; the outcome is made warp-uniform before any .sync.aligned op
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], phb, ctx));
                 if (!ok) break;
+                // the K block's MMAs are complete, so they have read the operand stage: warp 4
+                // hands it back to this CTA's producers
+                if (warp == 4 && lane == 0) mbar_arrive(&empty[it % STAGES]);
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sfa_full[j], (it / L::SFS) & 1, ctx));
                 if (!ok) break;
                 const float sa = sfa_ring[j * L::SF_SLOT + q * 32 + lane];
@@ -663,6 +722,62 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             }
             if (!ok) break;
             if (!ti.store) continue;
+            if (TAIL) {
+                // last-wave split. This warp's slice of a piece's partial: 32 rows x HALF columns,
+                // float4 c4 of lane l at [c4][l] (each store instruction writes 512 contiguous bytes)
+                constexpr int SLICE = 32 * HALF;                   // floats per warp slice
+                const int ticket = *ticket_smem;
+                const int r = t / p.tail_s;
+                const int piece = t - r * p.tail_s;
+                const int slot0 = r * (p.tail_s - 1) * (PAIR ? 2 : 1) + static_cast<int>(rank);
+                if (piece > 0) {
+                    const int slot = slot0 + (piece - 1) * (PAIR ? 2 : 1);
+                    float4 *dst = reinterpret_cast<float4 *>(p.ws + (static_cast<size_t>(slot) * 8 + mw) * SLICE);
+#pragma unroll
+                    for (int c4 = 0; c4 < HALF / 4; ++c4)
+                        __stcg(dst + c4 * 32 + lane,
+                               make_float4(acc[4 * c4], acc[4 * c4 + 1], acc[4 * c4 + 2], acc[4 * c4 + 3]));
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0 && !p.test_skip_tail) flag_store_release(p.flags + slot * 8 + mw, ticket);
+                    continue;
+                }
+                // piece 0: wait (bounded) for each later piece's slice, then add them in piece
+                // order, so that the sum does not depend on which piece finished first
+                bool got = true;
+                if (lane == 0) {
+                    const uint64_t t0 = globaltimer_ns();
+                    for (int pc = 1; pc < p.tail_s && got; ++pc) {
+                        const int slot = slot0 + (pc - 1) * (PAIR ? 2 : 1);
+                        while (flag_load_acquire(p.flags + slot * 8 + mw) != ticket) {
+                            if (*abort_flag) {
+                                got = false;
+                                break;
+                            }
+                            if (globaltimer_ns() - t0 > ctx->limit_ns) {
+                                report_error(ctx->err, ERR_TIMEOUT);
+                                *abort_flag = 1;
+                                got = false;
+                                break;
+                            }
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xFFFFFFFFu, got, 0);
+                if (!ok) break;
+                for (int pc = 1; pc < p.tail_s; ++pc) {
+                    const int slot = slot0 + (pc - 1) * (PAIR ? 2 : 1);
+                    const float4 *src = reinterpret_cast<const float4 *>(p.ws + (static_cast<size_t>(slot) * 8 + mw) * SLICE);
+#pragma unroll
+                    for (int c4 = 0; c4 < HALF / 4; ++c4) {
+                        const float4 v = __ldcg(src + c4 * 32 + lane);
+                        acc[4 * c4] += v.x;
+                        acc[4 * c4 + 1] += v.y;
+                        acc[4 * c4 + 2] += v.z;
+                        acc[4 * c4 + 3] += v.w;
+                    }
+                }
+            }
             if (KGRP) {
                 // fp32 D (a weight gradient): each thread stores its row's HALF columns, 16 bytes
                 // at a time, after adding C (read the same way; N % 16 == 0, so a 4-column
@@ -769,6 +884,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
 
     __syncwarp();                              // reconverge single-lane roles before the barrier
+    if (TAIL && p.tail_early) pdl_wait();
     tc_fence_before();
     if (PAIR)
         cluster_sync();
@@ -781,6 +897,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
         else
             tmem_dealloc(tmem_base, L::TMEM_COLS);
+    }
+    if (TAIL && threadIdx.x == 0) {
+        // the last CTA to finish publishes this launch's ticket as the epoch; the next launch
+        // on the stream reads it only after this grid has completed (griddepcontrol.wait)
+        __threadfence();
+        if (atomicAdd(p.epoch + 1, 1u) == gridDim.x - 1) {
+            p.epoch[1] = 0u;
+            p.epoch[0] = static_cast<unsigned>(*ticket_smem);
+            __threadfence();
+        }
     }
 #endif
 }

@@ -62,12 +62,6 @@ struct SwapParams {
     int one_issuer;   // experiments: warp 1 issues every K block (no second issuer)
 };
 
-// Ticket of a stream-K launch: one past the epoch word, never 0 (flags start out zero).
-__device__ __forceinline__ int streamk_ticket(const unsigned *epoch) {
-    const unsigned e = *reinterpret_cast<const volatile unsigned *>(epoch);
-    return static_cast<int>(e + 1u == 0u ? 1u : e + 1u);
-}
-
 template <int TN, int STAGES>
 struct SwapLayout {
     static_assert(TN == 64 || TN == 128, "token tile");

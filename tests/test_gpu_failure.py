@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 MODE = os.environ.get("DG_TEST_SKIP_RELEASE", "")
-CHILD = MODE in ("1", "2", "3")
+CHILD = MODE in ("1", "2", "3", "4")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -187,3 +187,36 @@ def test_child_streamk_timeout_then_exact(oracle):
     ref = oracle.gemm_nt(host(a), host(sfa), host(b), host(sfb), c)
     assert_close(bf16_host_f64(d_ws), ref, "stream-K after a flag timeout")
     assert torch.equal(d_static.view(torch.int16), d_ws.view(torch.int16))
+
+
+@pytest.mark.skipif(CHILD, reason="parent-process test")
+def test_tail_flag_wait_timeout_then_exact():
+    """A child process makes the piece CTAs of its first last-wave-split tile GEMM withhold their
+    partial flags (a debug-only switch), with a 100 ms wait limit: the first pieces' flag waits
+    run out and DG_ERR_TIMEOUT is reported; the next launch on the same workspace is exact."""
+    env = dict(os.environ, DG_TEST_SKIP_RELEASE="4", DG_WAIT_TIMEOUT_MS="100")
+    cmd = [sys.executable, "-m", "pytest", os.path.join(HERE, "test_gpu_failure.py"), "-q", "-x", "-m", "gpu",
+           "-k", "child"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    tail = "\n".join((r.stdout + r.stderr).splitlines()[-25:])
+    assert r.returncode == 0 and " passed" in r.stdout, tail
+
+
+@pytest.mark.skipif(MODE != "4", reason="runs in the child process of test_tail_flag_wait_timeout_then_exact")
+def test_child_tail_timeout_then_exact(oracle):
+    M, N, K = 512, 2048, 7168          # 16 pair tiles, each cut into pieces along K
+    x, w, c = synth.dense_inputs(M, N, K, True, salt=47)
+    x_bad, _, _ = synth.dense_inputs(M, N, K, False, salt=48)
+    b, sfb = ops.cast_per_block(bf16_dev(w))
+    a, sfa = ops.cast_per_token(bf16_dev(x))
+    a_bad, sfa_bad = ops.cast_per_token(bf16_dev(x_bad))   # other partials, so stale ones would show
+    cd = bf16_dev(c)
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+    ops.fp8_gemm_nt(a_bad, sfa_bad, b, sfb, cd)              # withholds its flags
+    assert "last-wave split" in _lib.dg_last_kernel()
+    d = ops.fp8_gemm_nt(a, sfa, b, sfb, cd)                 # no dg_get_device_error() in between
+    torch.cuda.synchronize()
+    assert _lib.dg_get_device_error() == _lib.DG_ERR_TIMEOUT
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+    ref = oracle.gemm_nt(host(a), host(sfa), host(b), host(sfb), c)
+    assert_close(bf16_host_f64(d), ref, "last-wave split after a flag timeout")
