@@ -526,6 +526,7 @@ class CudaArm:
             self.launch_cast(p, stream.cuda_stream)
             self.launch_gemm(p, stream.cuda_stream)
             p["kernel"] = self._lib.dg_last_kernel()
+            p["launches"] += self._lib.dg_last_launch_count() - 1   # a last-wave split adds one
         for _ in range(warmup):
             step(stream.cuda_stream)
         torch.cuda.synchronize(dev)

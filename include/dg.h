@@ -279,6 +279,11 @@ DG_API const char *dg_status_string(dg_status status);
  * benchmarks and profiles; valid until the thread's next GEMM call. */
 DG_API const char *dg_last_kernel(void);
 
+/* Number of kernels the calling thread's last launching GEMM call launched (0 before the
+ * first): 1, or 2 for a tile GEMM whose last-wave split ran behind a launch of the whole
+ * waves. For benchmarks that count launches. */
+DG_API int dg_last_launch_count(void);
+
 /* Bytes of device memory the library has allocated with cudaMalloc so far, over all devices
  * (the few-row stream-K workspaces); the static arrays of the module are not counted. */
 DG_API long long dg_allocated_bytes(void);

@@ -67,6 +67,7 @@ def load():
             "dg_fp8_gemm_tt": [P, P, P, P, P, P, I, I, I, P],
             "dg_k_grouped_fp8_gemm_tn_contiguous": [P, P, P, P, P, P, P, P, I, I, I, P],
             "dg_last_kernel": [],
+            "dg_last_launch_count": [],
             "dg_allocated_bytes": [],
         }
         for name, args in sig.items():
@@ -188,6 +189,11 @@ def dg_status_string(status: int) -> str:
 def dg_last_kernel() -> str:
     """Name of the GEMM kernel the calling thread's last GEMM call launched."""
     return load().dg_last_kernel().decode()
+
+
+def dg_last_launch_count() -> int:
+    """Number of kernels the calling thread's last GEMM call launched."""
+    return int(load().dg_last_launch_count())
 
 
 def dg_allocated_bytes() -> int:

@@ -39,6 +39,7 @@ std::atomic<long long> g_allocated{0};
 // Name of the GEMM kernel the calling thread's last GEMM call launched; dg_last_kernel().
 thread_local const char *t_last_kernel = "";
 thread_local char t_kernel_name[96];   // names with a number in them (the last-wave split)
+thread_local int t_last_launches = 0;  // kernels the thread's last GEMM call launched
 
 struct DeviceInfo {
     std::atomic<bool> ready{false};
@@ -499,6 +500,7 @@ dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p_in, int tiles,
                           PAIR ? "gemm_kernel (CTA pairs, last-wave split %d)" : "gemm_kernel (last-wave split %d)",
                           p.tail_s);
             t_last_kernel = t_kernel_name;
+            t_last_launches = p.tail_first > 0 ? 2 : 1;
             return r;
         }
     }
@@ -507,6 +509,7 @@ dg_status launch_gemm(const GemmMaps &mp, const dg::GemmParams &p_in, int tiles,
     cfg.gridDim = dim3(PAIR ? 2 * n_units : n_units, 1, 1);
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mp.a, mp.b, mp.sfa, mp.c, mp.d, mp.sfb, p);
     t_last_kernel = PAIR ? "gemm_kernel (CTA pairs)" : "gemm_kernel";
+    t_last_launches = 1;
     return from_cuda(e);
 }
 
@@ -713,6 +716,7 @@ dg_status launch_swap(const SwapMaps &mp, const dg::SwapParams &p, long long til
     if (grid <= 0) return DG_OK;
     Launch ln(dim3(static_cast<unsigned>(grid), 1, 1), dim3(L::THREADS, 1, 1), L::ALLOC, st);
     t_last_kernel = "gemm_swap_kernel (stream-K)";
+    t_last_launches = 1;
     return from_cuda(cudaLaunchKernelEx(&ln.cfg, kern, mp.w, mp.x, mp.sfa, mp.c, p));
 }
 
@@ -832,6 +836,7 @@ dg_status launch_splitk(const SwapMaps &mp, const dg::SwapParams &p, int tiles, 
     if (best_s == 0) return DG_ERR_UNSUPPORTED;
     Launch ln(dim3(static_cast<unsigned>(best_c * best_s), 1, 1), dim3(L::THREADS, 1, 1), L::ALLOC, st, best_s, true);
     t_last_kernel = "gemm_splitk_kernel (cluster split-K)";
+    t_last_launches = 1;
     return from_cuda(cudaLaunchKernelEx(&ln.cfg, kern, mp.w, mp.x, mp.sfa, p));
 }
 
@@ -941,6 +946,7 @@ dg_status run_gemm_ue8m0(const void *a, const uint32_t *sfa, const void *b, cons
     if (grid <= 0) return DG_OK;
     Launch ln(dim3(static_cast<unsigned>(grid), 1, 1), dim3(dg::BS_THREADS, 1, 1), dg::BsLayout::ALLOC, st);
     t_last_kernel = "gemm_bs_kernel (UE8M0 block-scaled MMA)";
+    t_last_launches = 1;
     return from_cuda(cudaLaunchKernelEx(&ln.cfg, dg::gemm_bs_kernel, tm_a, tm_b, p));
 }
 
@@ -1219,6 +1225,8 @@ dg_status dg_get_device_error(void *stream) {
 }
 
 const char *dg_last_kernel(void) { return t_last_kernel; }
+
+int dg_last_launch_count(void) { return t_last_launches; }
 
 long long dg_allocated_bytes(void) { return g_allocated.load(); }
 
