@@ -507,10 +507,16 @@ class CudaArm:
             l2 = "flush" if step_bytes < 512 * 2 ** 20 else "large"
         flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev) if l2 == "flush" else None
 
-        def step(sptr, ev=None):
+        # cold steps: an event pair inside the step graph brackets the work after the flush, so
+        # that the step time does not include the flushing write itself
+        fev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] if flush is not None else None
+
+        def step(sptr, ev=None, fe=None):
             if flush is not None:
                 flush.fill_(1)
             cur = torch.cuda.current_stream(dev)
+            if fe is not None:
+                fe[0].record(cur)
             for i, p in enumerate(probs):
                 if ev is not None:
                     ev[3 * i].record(cur)
@@ -520,6 +526,8 @@ class CudaArm:
                 self.launch_gemm(p, sptr)
                 if ev is not None:
                     ev[3 * i + 2].record(cur)
+            if fe is not None:
+                fe[1].record(cur)
 
         # eager warm-up, which also names the kernel each problem takes
         for p in probs:
@@ -544,7 +552,7 @@ class CudaArm:
             step(cap.cuda_stream)                                 # warm the capture stream
             torch.cuda.synchronize(dev)
             with torch.cuda.graph(g_step, stream=cap):
-                step(cap.cuda_stream)
+                step(cap.cuda_stream, fe=fev)
             with torch.cuda.graph(g_ev, stream=cap):
                 step(cap.cuda_stream, evs)
         torch.cuda.synchronize(dev)
@@ -555,14 +563,19 @@ class CudaArm:
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(dev)
         torch.cuda.synchronize(dev)
+        work_ms = []
         with ClockSampler(local_rank) as clk:
             start.record(stream)
             for _ in range(steps):
                 g_step.replay()
+                if fev is not None:                               # cold: read each step's pair
+                    torch.cuda.synchronize(dev)
+                    work_ms.append(fev[0].elapsed_time(fev[1]))
             end.record(stream)
             torch.cuda.synchronize(dev)
         barrier(dev)
-        local_ms = start.elapsed_time(end) / steps
+        with_flush_ms = start.elapsed_time(end) / steps
+        local_ms = statistics.fmean(work_ms) if work_ms else with_flush_ms
         if self._lib.dg_get_device_error(stream.cuda_stream) != 0:
             raise RuntimeError("device error word set during the timed region")
         cast_t = [[] for _ in probs]
@@ -574,12 +587,15 @@ class CudaArm:
                 cast_t[i].append(evs[3 * i].elapsed_time(evs[3 * i + 1]))
                 gemm_t[i].append(evs[3 * i + 1].elapsed_time(evs[3 * i + 2]))
         del g_step, g_ev
-        return dict(local_ms=local_ms, cast_ms=[statistics.fmean(v) for v in cast_t],
+        return dict(local_ms=local_ms, with_flush_ms=with_flush_ms if work_ms else None,
+                    cast_ms=[statistics.fmean(v) for v in cast_t],
                     gemm_ms=[statistics.fmean(v) for v in gemm_t], clocks=clk.summary(), l2=l2,
                     launches_per_step=sum(p["launches"] for p in probs) + (1 if flush is not None else 0))
 
 
-L2_TEXT = {"flush": "256 MB L2-flushing write at the start of every step (cold weights)",
+L2_TEXT = {"flush": "256 MB L2-flushing write at the start of every step (cold weights); the step time is "
+                    "taken by an event pair inside the step graph after the flush, so it excludes the flushing "
+                    "write (ms_per_step_with_flush includes it)",
            "warm": "no flush: steps back to back (weights partly L2-resident)",
            "large": "no flush: one step's working set is far above the 126 MB L2"}
 
@@ -735,6 +751,8 @@ def run_cuda(args):
             sroof, spp = roofline_of(sprobs, st, name if l2 != "warm" else key)
             subs[key] = {"workload": swl["desc"], "value": round(sflops / (sms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                          "ms_per_step": round(sms, 4), "steps": args.sub_steps, "l2": L2_TEXT[st["l2"]],
+                         "ms_per_step_with_flush": (round(reduce_max(st["with_flush_ms"], device), 4)
+                                                    if st["with_flush_ms"] is not None else None),
                          "gpu_launches": st["launches_per_step"] * args.sub_steps,
                          "roofline": sroof, "per_problem": spp, "clocks": st["clocks"]}
             for p in sprobs:

@@ -11,29 +11,32 @@
 // Scales in global memory (packed, MN-major for A): sfa uint32 [ceil(Kb/4)][pad4(M)], byte kb%4
 // of word (kb/4, m) = the UE8M0 of A[m, kb·128 ..]; sfb uint32 [Nb][ceil(Kb/4)] for the 128x128
 // blocks of B. The MMA reads its scales from TMEM: per K block (four MMAs of K = 32, one scale
-// per row of A and per row of B for each), the scales go to TMEM by tcgen05.cp from "scale
-// atoms" in shared memory: 512 bytes for 128 rows x 4 K sub-blocks, row r's byte for sub-block
-// j at 16·(r%32) + 4·(r/32) + j. tcgen05.cp .32x128b.warpx4 puts atom row l into TMEM lane l
-// (columns c .. c+3) of all four lane quadrants; the MMA then finds row r's scale in lane r%32,
-// column c + r/32, byte j (the scale-factor id of the instruction descriptor). With 1x128 and
-// 128x128 scale blocks the four bytes of a row are equal, so every sub-block sees the same scale.
+// per row of A and per row of B for each), row r of A's scale sits in TMEM lane r%32, column
+// c + r/32, byte j (the scale-factor id of the instruction descriptor picks the byte), the same
+// in all four lane quadrants, and B's likewise in columns c+4 .. c+11 (rows 0-127, 128-255) —
+// the layout a tcgen05.cp .32x128b.warpx4 of a 512-byte scale atom gives. The scale warps write
+// it directly from registers with tcgen05.st, each warp its own lane quadrant. With 1x128 and
+// 128x128 scale blocks the four bytes of a word are equal, so every sub-block sees the same scale.
 //
 // Tiles: one CTA per 128 x BN tile (cta_group::1, M = 128, N = BN = 224), persistent. Two TMEM
 // accumulators of 224 columns (448 of the 512) let a tile's epilogue overlap the next tile's
-// MMAs; the last 64 columns hold four 16-column scale slots (SFA 4 columns, SFB 8 columns for
-// the up to 256 B rows of two 128-row atoms), one per ring stage.
+// MMAs; the last 64 columns hold four 16-column scale slots, a ring of its own beside the five
+// operand stages.
 //
 // CTA layout (384 threads): warp 0 A producers and warp 2 B producers (lanes 0 and 16: even and
-// odd K blocks, TMA into a STAGES-deep ring), warp 1 TMEM allocator and the MMA issuer (one
-// thread: copies the stage's scale atoms to TMEM, issues four block-scaled MMAs, commits the
-// stage every two K blocks and the accumulator at the tile's end), warps 4-7 the scale-atom
-// writers (per K block they unpack the stage's scale bytes into its atoms once the stage's
-// previous MMAs are done, running up to the ring's depth ahead of the MMA), warps 8-11 the
-// epilogue (per tile they read the accumulator with tcgen05.ld, release it, add C and store D
-// as bf16, rounded to nearest even, while the MMA already works on the next tile).
+// odd K blocks, TMA into a 5-deep ring), warp 1 TMEM allocator and the MMA issuer (one thread:
+// four block-scaled MMAs per K block, a commit of the stages every two K blocks and of the
+// accumulator at the tile's end), warps 4-7 the scale writers (per K block, once the MMAs that
+// last used the slot are done, they load the packed scale words, unpack the K block's byte and
+// store the slot with tcgen05.st), warps 8-11 the epilogue (per tile, 64 columns at a time: C
+// loads issued, the accumulator read with tcgen05.ld, released after its last columns, C
+// added and D stored as bf16, rounded to nearest even, while the MMA already works on the next
+// tile).
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "dg_gemm.cuh"
 #include "dg_ptx.cuh"
@@ -41,10 +44,11 @@
 namespace dg {
 
 constexpr int BS_BN = 224;                 // tile columns (two accumulators + scale slots fit 512 TMEM columns)
-constexpr int BS_STAGES = 4;
+constexpr int BS_STAGES = 5;
+constexpr int BS_SF_SLOTS = 4;             // TMEM scale slots, a ring of their own
 constexpr int BS_THREADS = 384;
 constexpr int BS_SF_COL0 = 2 * BS_BN;      // first TMEM column of the scale slots (448)
-constexpr int BS_SF_SLOT_COLS = 16;        // per stage: SFA 4 columns, SFB 8 columns
+constexpr int BS_SF_SLOT_COLS = 16;        // per slot: SFA 4 columns, SFB 8 columns
 
 struct BsParams {
     int M, N, K;
@@ -64,19 +68,17 @@ struct BsParams {
 struct BsLayout {
     static constexpr int A_BYTES = BM * BK;                  // 16 KB
     static constexpr int B_BYTES = BS_BN * BK;               // 28 KB
-    static constexpr int ATOM = 512;                         // 128 rows x 4 scale bytes
-    static constexpr int SF_BYTES = 3 * ATOM;                // SFA + two SFB atoms per stage
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + BS_STAGES * A_BYTES;
-    static constexpr int OFF_SF = OFF_B + BS_STAGES * B_BYTES;
-    static constexpr int OFF_BAR = OFF_SF + BS_STAGES * SF_BYTES;
-    // full, empty, sf_full per stage; tfull, tempty per accumulator
-    static constexpr int NUM_BARS = 3 * BS_STAGES + 4;
+    static constexpr int OFF_BAR = OFF_B + BS_STAGES * B_BYTES;
+    // full, empty per stage; sf_full per scale slot; tfull, tempty per accumulator
+    static constexpr int NUM_BARS = 2 * BS_STAGES + BS_SF_SLOTS + 4;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int BYTES = OFF_MISC + static_cast<int>(sizeof(WaitCtx));
     static constexpr int ALLOC = BYTES + 1024;
     static constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
-    static_assert(OFF_B % 1024 == 0 && OFF_SF % 1024 == 0, "1024-byte aligned operand tiles");
+    static_assert(OFF_B % 1024 == 0, "1024-byte aligned operand tiles");
+    static_assert(BS_SF_COL0 + BS_SF_SLOTS * BS_SF_SLOT_COLS <= 512, "TMEM columns");
     static_assert(ALLOC <= 232448, "shared memory budget");
 };
 
@@ -101,24 +103,6 @@ __device__ __forceinline__ void umma_mxf8_bs(uint32_t d_tmem, uint64_t adesc, ui
         : "memory");
 }
 
-// Shared-memory descriptor of a scale atom for tcgen05.cp: 32 rows of 16 bytes, no swizzle,
-// K-major core matrices of 8 rows x 16 bytes (128 bytes) one after another (stride byte offset
-// 128), version 1, layout type 0.
-__device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-    d |= static_cast<uint64_t>(16 >> 4) << 16;
-    d |= static_cast<uint64_t>(128 >> 4) << 32;
-    d |= static_cast<uint64_t>(1) << 46;
-    return d;
-}
-
-// 32 lanes x 128 bits from shared memory into TMEM columns taddr .. taddr+3 of all four lane
-// quadrants (the copy of a scale atom).
-__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
 __global__ void __launch_bounds__(BS_THREADS, 1)
     gemm_bs_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                    const BsParams p) {
@@ -129,8 +113,8 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
     uint64_t *empty = full + S;
-    uint64_t *sf_full = empty + S;
-    uint64_t *tfull = sf_full + S;
+    uint64_t *sf_full = empty + S;            // [BS_SF_SLOTS]
+    uint64_t *tfull = sf_full + BS_SF_SLOTS;
     uint64_t *tempty = tfull + 2;
     WaitCtx *ctx = reinterpret_cast<WaitCtx *>(smem + L::OFF_MISC);
     volatile int *abort_flag = &ctx->abort;
@@ -142,8 +126,8 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&sf_full[s], 4);         // one arrive per atom-writing warp
         }
+        for (int j = 0; j < BS_SF_SLOTS; ++j) mbar_init(&sf_full[j], 4);   // one arrive per scale warp
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 4);          // one arrive per epilogue warp
@@ -192,7 +176,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
                 }
             }
         } else if (warp == 1 && lane == 0) {
-            // MMA issuer. The stage's scale atoms go to its TMEM scale slot, then four MMAs of
+            // MMA issuer. Once the stage is loaded and its scale slot written, four MMAs of
             // K = 32; a commit releases two stages at a time (a commit holds back this thread's
             // later MMAs until the committed ones are done, so fewer commits keep the pipe full)
             uint32_t it = 0, tcount = 0;
@@ -206,14 +190,12 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
                 int pending = 0;
                 for (int kb = 0; kb < p.Kb; ++kb, ++it) {
                     const int s = it % S;
-                    ok = mbar_wait(&full[s], (it / S) & 1, ctx) && mbar_wait(&sf_full[s], (it / S) & 1, ctx);
+                    const int j = it % BS_SF_SLOTS;
+                    ok = mbar_wait(&full[s], (it / S) & 1, ctx) &&
+                         mbar_wait(&sf_full[j], (it / BS_SF_SLOTS) & 1, ctx);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t sf_col = tmem_base + static_cast<uint32_t>(BS_SF_COL0 + s * BS_SF_SLOT_COLS);
-                    const uint32_t sf_smem = smem_u32(smem + L::OFF_SF + s * L::SF_BYTES);
-                    tmem_cp_32x128b_x4(sf_col, sdesc_sf_atom(sf_smem));                      // SFA
-                    tmem_cp_32x128b_x4(sf_col + 4, sdesc_sf_atom(sf_smem + L::ATOM));        // SFB rows 0-127
-                    tmem_cp_32x128b_x4(sf_col + 8, sdesc_sf_atom(sf_smem + 2 * L::ATOM));    // SFB rows 128-255
+                    const uint32_t sf_col = tmem_base + static_cast<uint32_t>(BS_SF_COL0 + j * BS_SF_SLOT_COLS);
                     const uint64_t ad = sdesc_k_sw128(smem_u32(smem + L::OFF_A + s * L::A_BYTES));
                     const uint64_t bd = sdesc_k_sw128(smem_u32(smem + L::OFF_B + s * L::B_BYTES));
 #pragma unroll
@@ -230,41 +212,60 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
             }
         }
     } else if (warp < 8) {
-        // ---------------- scale atoms (warps 4-7): thread r writes row r of every atom ----------------
-        const int r = threadIdx.x - 128;           // 0..127
+        // ---------------- scales (warps 4-7) into the TMEM scale slots ----------------
+        // Warp q (= warp % 4) writes TMEM lanes 32q..32q+31 of slot j = it % BS_SF_SLOTS, all four
+        // quadrants alike (the layout a 32x128b.warpx4 copy of a scale atom would give): lane l,
+        // column c + k holds the UE8M0 of A row 32k + l of the tile (its byte repeated for the
+        // four K sub-blocks), column c + 4 + 4h + k that of B row 128h + 32k + l (the scale of its
+        // 128x128 block). A slot is rewritten once the MMAs of the K block that last used it are
+        // done (their stage's release; the ring of stages is longer than the ring of slots).
+        const int q = warp & 3;
         uint32_t it = 0;
         bool ok = true;
         for (int t = cid; t < p.num_tiles && ok; t += ncid) {
             int mb, nbk;
             tile_of(t, mb, nbk);
-            const int row = mb * BM + r;
             for (int kb = 0; kb < p.Kb; ++kb, ++it) {
-                const int s = it % S;
-                // the stage's previous MMAs have read its atoms (their commit released the stage)
-                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], ((it / S) & 1) ^ 1, ctx));
-                if (!ok) break;
-                uint32_t *atoms = reinterpret_cast<uint32_t *>(smem + L::OFF_SF + s * L::SF_BYTES);
-                const int shift = 8 * (kb & 3);
-                const int slot = 4 * (r & 31) + (r >> 5);
-                // SFA: row r's byte, replicated over the four K sub-blocks
-                const uint32_t wa = row < p.M ? __ldg(p.sfa + static_cast<size_t>(kb >> 2) * p.ld_sfa + row) : 0x7F7F7F7Fu;
-                atoms[slot] = ((wa >> shift) & 0xFFu) * 0x01010101u;
-                // SFB: B rows r and 128 + r of the tile (rows past its 224 are never read) take
-                // the scale of their 128x128 block
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int n = nbk * BS_BN + h * 128 + r;
-                    const int nb = min(n, p.N - 1) >> 7;
-                    const uint32_t wb = __ldg(p.sfb + static_cast<size_t>(nb) * p.Kq + (kb >> 2));
-                    atoms[128 * (1 + h) + slot] = ((wb >> shift) & 0xFFu) * 0x01010101u;
+                const int j = it % BS_SF_SLOTS;
+                if (it >= static_cast<uint32_t>(BS_SF_SLOTS)) {
+                    const uint32_t prev = it - BS_SF_SLOTS;
+                    ok = __all_sync(0xFFFFFFFFu, mbar_wait(&empty[prev % S], (prev / S) & 1, ctx));
+                    if (!ok) break;
+                    tc_fence_after();
                 }
-                fence_proxy_async_smem();          // generic writes -> the tensor core's copy
+                const int shift = 8 * (kb & 3);
+                uint32_t wa[4], wb[8];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int row = mb * BM + 32 * k + lane;
+                    const uint32_t w = row < p.M ? __ldg(p.sfa + static_cast<size_t>(kb >> 2) * p.ld_sfa + row) : 0x7F7F7F7Fu;
+                    wa[k] = ((w >> shift) & 0xFFu) * 0x01010101u;
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int n = nbk * BS_BN + 128 * h + 32 * k + lane;   // rows past the tile's 224 are never read
+                        const int nb = min(n, p.N - 1) >> 7;
+                        const uint32_t w = __ldg(p.sfb + static_cast<size_t>(nb) * p.Kq + (kb >> 2));
+                        wb[4 * h + k] = ((w >> shift) & 0xFFu) * 0x01010101u;
+                    }
+                const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                      static_cast<uint32_t>(BS_SF_COL0 + j * BS_SF_SLOT_COLS);
+                tmem_st4(tcol, wa);
+                tmem_st8(tcol + 4, wb);
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
-                if ((r & 31) == 0) mbar_arrive(&sf_full[s]);
+                if (lane == 0) mbar_arrive(&sf_full[j]);
             }
         }
     } else {
         // ---------------- epilogue (warps 8-11): lanes 32q.., all 224 columns ----------------
+        // Per tile: this thread's row of C is prefetched into L2 before the accumulator is ready;
+        // then 64 columns at a time (the last group 32): the C loads of the group are issued,
+        // its TMEM loads issued and waited for, and the sums stored, so that every memory and
+        // TMEM latency of a group overlaps the others of the same group.
         const int q = warp & 3;                    // TMEM lane quadrant
         uint32_t tcount = 0;
         bool ok = true;
@@ -272,50 +273,66 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
             int mb, nbk;
             tile_of(t, mb, nbk);
             const int b = tcount & 1;
+            const int row = mb * BM + q * 32 + lane;
+            const int col0 = nbk * BS_BN;
+            const size_t rbase = static_cast<size_t>(row < p.M ? row : 0) * p.N;
+
             ok = __all_sync(0xFFFFFFFFu, mbar_wait(&tfull[b], (tcount >> 1) & 1, ctx));
             if (!ok) break;
             tc_fence_after();
-            const int row = mb * BM + q * 32 + lane;
-            const int col0 = nbk * BS_BN;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BS_BN);
-            const size_t rbase = static_cast<size_t>(row < p.M ? row : 0) * p.N;
-#pragma unroll 1
-            for (int c = 0; c < BS_BN / 16; ++c) {
-                uint32_t r16[16];
-                tmem_ld16(taddr + c * 16, r16);
-                tmem_ld_wait();
-                if (c + 1 == BS_BN / 16) {
+            // NC chunks of 16 columns starting at chunk c0 (N % 16 == 0: a chunk is all in or out)
+            auto group = [&](auto nc_tag, int c0) {
+                constexpr int NC = decltype(nc_tag)::value;
+                uint4 cv[NC][2];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    const int col = col0 + (c0 + c) * 16;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                        cv[c][hh] = p.has_c && row < p.M && col < p.N
+                                        ? __ldg(reinterpret_cast<const uint4 *>(p.c + rbase + col + hh * 8))
+                                        : make_uint4(0, 0, 0, 0);
+                }
+                uint32_t r16[NC][16];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) tmem_ld16(taddr + (c0 + c) * 16, r16[c]);
+#pragma unroll
+                for (int c = 0; c < NC; ++c) tmem_ld_wait_regs16(r16[c]);
+                if (c0 + NC == BS_BN / 16) {
                     // every column of the accumulator is in registers: the next tile may use it
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&tempty[b]);
                 }
-                const int col = col0 + c * 16;
-                if (row < p.M && col < p.N) {      // N % 16 == 0: a 16-column chunk is all in or out
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        float f[8];
+                for (int c = 0; c < NC; ++c) {
+                    const int col = col0 + (c0 + c) * 16;
+                    if (row < p.M && col < p.N) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r16[hh * 8 + e]);
-                        if (p.has_c) {
-                            const uint4 cv = __ldg(reinterpret_cast<const uint4 *>(p.c + rbase + col + hh * 8));
-                            const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint32_t cw[4] = {cv[c][hh].x, cv[c][hh].y, cv[c][hh].z, cv[c][hh].w};
+                            uint32_t w[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                f[2 * e] += __uint_as_float(cw[e] << 16);
-                                f[2 * e + 1] += __uint_as_float(cw[e] & 0xFFFF0000u);
+                                float f0 = __uint_as_float(r16[c][hh * 8 + 2 * e]);
+                                float f1 = __uint_as_float(r16[c][hh * 8 + 2 * e + 1]);
+                                if (p.has_c) {
+                                    f0 += __uint_as_float(cw[e] << 16);
+                                    f1 += __uint_as_float(cw[e] & 0xFFFF0000u);
+                                }
+                                __nv_bfloat162 h2 = __floats2bfloat162_rn(f0, f1);
+                                w[e] = *reinterpret_cast<uint32_t *>(&h2);
                             }
+                            *reinterpret_cast<uint4 *>(p.d + rbase + col + hh * 8) = make_uint4(w[0], w[1], w[2], w[3]);
                         }
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            __nv_bfloat162 h2 = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
-                            w[e] = *reinterpret_cast<uint32_t *>(&h2);
-                        }
-                        *reinterpret_cast<uint4 *>(p.d + rbase + col + hh * 8) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
-            }
+            };
+            static_assert(BS_BN % 64 == 32, "three groups of 64 columns and one of 32");
+#pragma unroll 1
+            for (int g = 0; g < BS_BN / 64; ++g) group(std::integral_constant<int, 4>(), g * 4);
+            group(std::integral_constant<int, 2>(), (BS_BN / 64) * 4);
         }
     }
 

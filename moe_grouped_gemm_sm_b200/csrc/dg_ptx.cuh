@@ -349,6 +349,40 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// tcgen05.wait::ld, then 16 loaded registers read in the same asm statement (separate in and
+// out operands), so that no use of them can be scheduled above the wait.
+__device__ __forceinline__ void tmem_ld_wait_regs16(uint32_t (&r)[16]) {
+    uint32_t t[16];
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;\n\t"
+        "mov.b32 %0, %16;\n\tmov.b32 %1, %17;\n\tmov.b32 %2, %18;\n\tmov.b32 %3, %19;\n\t"
+        "mov.b32 %4, %20;\n\tmov.b32 %5, %21;\n\tmov.b32 %6, %22;\n\tmov.b32 %7, %23;\n\t"
+        "mov.b32 %8, %24;\n\tmov.b32 %9, %25;\n\tmov.b32 %10, %26;\n\tmov.b32 %11, %27;\n\t"
+        "mov.b32 %12, %28;\n\tmov.b32 %13, %29;\n\tmov.b32 %14, %30;\n\tmov.b32 %15, %31;"
+        : "=r"(t[0]), "=r"(t[1]), "=r"(t[2]), "=r"(t[3]), "=r"(t[4]), "=r"(t[5]), "=r"(t[6]), "=r"(t[7]),
+          "=r"(t[8]), "=r"(t[9]), "=r"(t[10]), "=r"(t[11]), "=r"(t[12]), "=r"(t[13]), "=r"(t[14]), "=r"(t[15])
+        : "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = t[i];
+}
+
+// 32 lanes x 32 bits, 4 / 8 consecutive columns from registers into TMEM: thread t of the warp
+// writes TMEM lane (lane field of taddr) + t, columns col .. col+3 / col+7. Complete after
+// tcgen05.wait::st.
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Register budget hand-off between warpgroups (all threads of a warpgroup execute it).
 template <int N>
 __device__ __forceinline__ void reg_alloc() {
