@@ -2,6 +2,7 @@
 declares; host-side helpers that need no device behave as documented."""
 import ctypes
 import subprocess
+import threading
 
 import pytest
 
@@ -36,6 +37,41 @@ def test_host_only_helpers(lib):
     assert [_lib.dg_sf_ld(x) for x in (0, 1, 4, 5, 4093)] == [0, 4, 4, 8, 4096]
     for code, name in _lib.STATUS.items():
         assert _lib.dg_status_string(code) == name
+
+
+def test_last_call_reporting_starts_empty(lib):
+    """dg_last_kernel / dg_last_launch_count are per thread: a thread that made no GEMM call
+    sees the empty name and a count of 0."""
+    seen = {}
+
+    def probe():
+        seen["name"] = _lib.dg_last_kernel()
+        seen["launches"] = _lib.dg_last_launch_count()
+    t = threading.Thread(target=probe)
+    t.start()
+    t.join()
+    assert seen == {"name": "", "launches": 0}
+
+
+def test_newer_entry_points_reject_bad_arguments_without_a_device(lib):
+    P = 16
+    ks = (ctypes.c_int * 2)(128, 256)
+    bad_ks = (ctypes.c_int * 2)(128, 100)
+    kg = lib.dg_k_grouped_fp8_gemm_tn_contiguous
+    assert kg(P, P, P, P, None, P, ks, P, 2, 64, 136, None) == _lib.DG_ERR_INVALID_ARG      # N % 16
+    assert kg(P, P, P, P, None, P, ks, P, 2, 72, 128, None) == _lib.DG_ERR_INVALID_ARG      # M % 16
+    assert kg(P, P, P, P, None, P, bad_ks, P, 2, 64, 128, None) == _lib.DG_ERR_INVALID_ARG  # K group % 128
+    assert kg(P, P, P, P, None, P, ks, P, 0, 64, 128, None) == _lib.DG_ERR_INVALID_ARG      # G = 0
+    assert kg(P, P, P, P, None, P, ks, P, 512, 64, 128, None) == _lib.DG_ERR_INVALID_ARG    # G > 511
+    assert kg(P, P, P, P, None, P + 4, ks, P, 2, 64, 128, None) == _lib.DG_ERR_ALIGNMENT
+    assert kg(P, P, P, P, None, P, ks, P, 2, 0, 128, None) == _lib.DG_OK                     # empty
+    assert lib.dg_fp8_gemm_nt_ue8m0(P, P, P, P, None, P, 64, 136, 128, None) == _lib.DG_ERR_INVALID_ARG
+    assert lib.dg_fp8_gemm_nt_ue8m0(P, P, P, P, None, P, 0, 128, 128, None) == _lib.DG_OK
+    assert lib.dg_fp8_gemm_nn(P, P, P, P, None, P, 64, 136, 128, None) == _lib.DG_ERR_INVALID_ARG   # B MN-major: N % 16
+    assert lib.dg_fp8_gemm_tn(P, P, P, P, None, P, 72, 128, 128, None) == _lib.DG_ERR_INVALID_ARG   # A MN-major: M % 16
+    assert lib.dg_fp8_gemm_tt(P, P, P, P, None, P, 72, 136, 128, None) == _lib.DG_ERR_INVALID_ARG
+    assert lib.dg_fp8_gemm_tt(P, P, P, P, None, P, 0, 128, 128, None) == _lib.DG_OK
+    assert lib.dg_fp8_gemm_nt_noalloc(P, P, P, P, None, P, 64, 128, 100, None) == _lib.DG_ERR_INVALID_ARG
 
 
 def test_argument_errors_need_no_device(lib):

@@ -103,6 +103,17 @@ def test_masked_small(oracle, G, M_max, N, K, lo, hi, with_c):
     check_masked(oracle, masked_m, dv, hv, G, M_max, N, 192, f"masked G={G} N={N} K={K}")
 
 
+@pytest.mark.parametrize("expected_m,kernel", [(32, "gemm_kernel"), (128, "gemm_kernel"),
+                                               (192, "gemm_kernel (CTA pairs)"), (0, "gemm_kernel (CTA pairs)")])
+def test_masked_expected_m_picks_the_tile(oracle, expected_m, kernel):
+    """expected_m <= 128 takes 128-row tiles, above it 256-row CTA-pair tiles (0: M_max decides);
+    both give the oracle's result on the same experts, and rows >= masked_m keep the sentinel."""
+    G, M_max, N, K = 6, 256, 520, 384
+    masked_m, dv, hv = masked_case(oracle, G, M_max, N, K, 0, 256, True, salt=61)
+    check_masked(oracle, masked_m, dv, hv, G, M_max, N, expected_m, f"masked expected_m={expected_m}")
+    assert _lib.dg_last_kernel() == kernel
+
+
 def test_masked_edge_counts(oracle):
     """masked_m of 0, 1, 31, 32, 33, 127, 128, 129 and M_max: partial warp slabs and tiles."""
     G, M_max, N, K = 9, 160, 264, 256
