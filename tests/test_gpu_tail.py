@@ -84,6 +84,22 @@ def test_tail_split_deterministic():
 
 
 @pytest.mark.skipif(bool(CHILD), reason="parent-process test")
+def test_tail_split_c_aliases_d(oracle):
+    """C passed as D: the last-wave pieces read C of their own tiles only, which the launch of the
+    whole waves, running beside them, never writes."""
+    M, N, K = 4096, 1280, 8192
+    dv, c = operands(M, N, K, True, salt=8)
+    a, sfa, b, sfb, cd = dv
+    d = cd.clone()
+    ops.fp8_gemm_nt(a, sfa, b, sfb, d, out=d)
+    torch.cuda.synchronize()
+    assert "last-wave split" in _lib.dg_last_kernel()
+    assert _lib.dg_get_device_error() == _lib.DG_OK
+    ref = oracle.gemm_nt(host(a), host(sfa), host(b), host(sfb), c)
+    assert_close(bf16_host_f64(d), ref, "last-wave split with C aliasing D")
+
+
+@pytest.mark.skipif(bool(CHILD), reason="parent-process test")
 def test_tail_split_under_graph_replay():
     """Captured into a CUDA graph after the stream's workspace exists, the split GEMM replays
     with the launch tickets advancing replay after replay: same bits as the eager call."""
