@@ -115,6 +115,7 @@ struct GemmParams {
 template <int BN, int STAGES, bool PAIR, bool PAIR_LIST, bool KGRP = false>
 struct GemmLayout {
     static_assert(BN % 128 == 0 && BN <= 256, "BN must be 128 or 256");
+    static_assert(BN / 2 / 32 >= 2, "the TMEM release sits after the second-to-last 32-column batch");
     static constexpr int HALF = BN / 2;                      // columns per math warpgroup
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;        // rows of B loaded by one CTA
     static constexpr int A_BYTES = BM * BK;
@@ -703,21 +704,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         acc[c * 32 + 2 * i + 1] = a2.y;
                     }
                     if (c + 1 < HALF / 32) tmem_ld_wait_regs32(r[(c + 1) & 1]);
+                    if (c + 2 == HALF / 32) {
+                        // the last batch is in registers: every TMEM read of the buffer is complete
+                        // (wait::ld) and sa was consumed, so the buffer goes back to the MMA before
+                        // the last batch is folded in; a relaxed arrive suffices. (A failure test
+                        // can withhold one release: the MMA's bounded wait then runs out.)
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0 && !(p.test_skip_release && blockIdx.x == 0 && warp == 4 && it == 0)) {
+                            if (PAIR)
+                                mbar_arrive_cluster_relaxed(tempty_leader0 + b * 8);
+                            else
+                                mbar_arrive_relaxed(&tempty[b]);
+                        }
+                    }
                 }
                 if (KGRP) {                            // the column scales are read too
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_relaxed(&sfa_empty[j]);
-                }
-                tc_fence_before();
-                __syncwarp();
-                // TMEM reads are complete (wait::ld) and sa was consumed: a relaxed arrive suffices.
-                // (A failure test can withhold one release: the MMA's bounded wait then runs out.)
-                if (lane == 0 && !(p.test_skip_release && blockIdx.x == 0 && warp == 4 && it == 0)) {
-                    if (PAIR)
-                        mbar_arrive_cluster_relaxed(tempty_leader0 + b * 8);
-                    else
-                        mbar_arrive_relaxed(&tempty[b]);
                 }
             }
             if (!ok) break;
