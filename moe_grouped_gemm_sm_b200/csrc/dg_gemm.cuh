@@ -39,7 +39,8 @@
 //   warps 4-11  two math warpgroups. Warp w reads TMEM lanes 32·(w%4)..+31 (its 32 rows);
 //               warpgroup j owns columns [j·BN/2, (j+1)·BN/2). Per K block: wait for the TMEM
 //               buffer, load the partial in 32-column batches (the next batch in flight while
-//               the previous one is folded in), release the buffer, acc = fma(p, sa·sb, acc).
+//               the previous one is folded in as acc = fma(p, sa·sb, acc)), and release the
+//               buffer as soon as the last batch is in registers, before it is folded in.
 //               sfa arrives by TMA in a ring of its own (one BM-float column per K block,
 //               loaded by the producer ahead of the operands), sfb one 32-K-block window per
 //               lane broadcast by shuffle. Epilogue: C (prefetched by TMA at tile start) is added, the
